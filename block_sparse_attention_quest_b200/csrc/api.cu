@@ -1,0 +1,320 @@
+// C ABI of libresa: argument validation, workspace layout, launch plans.
+// Declarations and the meaning of every argument are in include/resa.h.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "../../include/resa.h"
+#include "launch.h"
+
+using namespace resa;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+// upper bound on co-resident CTAs assumed when sizing split partials
+constexpr int kSplitCtaBound = 1024;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int num_sms = 0;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev[dev].num_sms == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    g_dev[dev].num_sms = n;
+  }
+  return g_dev[dev].num_sms;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return g_encode;
+}
+
+// 2-D view [B*H*L_max rows][D cols] of a bf16 cache, 16 x 64 boxes, 128-byte swizzle
+bool make_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(s.D),
+                        static_cast<cuuint64_t>(s.B) * s.H * static_cast<cuuint64_t>(s.L_max)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(s.D) * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int check_dims(const resa_dims* d, Shape* s) {
+  if (d == nullptr) return RESA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_kv_heads < 1 || d->n_q_heads < 1 || d->max_len < 16 ||
+      d->max_len % 16 != 0)
+    return RESA_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads != 0) return RESA_ERR_INVALID_ARG;
+  if (d->dtype != RESA_F32 && d->dtype != RESA_BF16) return RESA_ERR_INVALID_ARG;
+  if (d->block_size != 16) return RESA_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return RESA_ERR_UNSUPPORTED;
+  const int G = d->n_q_heads / d->n_kv_heads;
+  if (G > 8) return RESA_ERR_UNSUPPORTED;
+  // TMA row coordinates are signed 32-bit
+  const double rows = static_cast<double>(d->batch) * d->n_kv_heads * static_cast<double>(d->max_len);
+  if (rows >= 2147483648.0) return RESA_ERR_UNSUPPORTED;
+  // grid.y / grid.z limits
+  if (d->n_kv_heads > 65535 || static_cast<int64_t>(d->batch) * 1024 > 65535 * 1024LL)
+    return RESA_ERR_UNSUPPORTED;
+  s->B = d->batch;
+  s->Hq = d->n_q_heads;
+  s->H = d->n_kv_heads;
+  s->G = G;
+  s->D = d->head_dim;
+  s->L_max = d->max_len;
+  s->Mmax = static_cast<int>(d->max_len / 16);
+  s->bf16 = d->dtype == RESA_BF16;
+  return RESA_OK;
+}
+
+int64_t blocks_of(int64_t len) { return (len + 15) / 16; }
+
+int splits_for(int units, int64_t min_blocks, int num_sms, const Shape& s) {
+  const int target = num_sms * attend_ctas_per_sm(s);
+  int S = units >= target ? 1 : target / units;
+  const int bound = units >= kSplitCtaBound ? 1 : kSplitCtaBound / units;
+  if (S > bound) S = bound;
+  if (S > kMaxSplits) S = kMaxSplits;
+  if (S > min_blocks) S = static_cast<int>(min_blocks);
+  return S < 1 ? 1 : S;
+}
+
+// bound used for workspace sizing (independent of the device)
+int64_t split_bound(int64_t units) {
+  int64_t S = units >= kSplitCtaBound ? 1 : kSplitCtaBound / units;
+  return S > kMaxSplits ? kMaxSplits : S;
+}
+
+struct WsLayout {
+  size_t scores, sel, part_ml, part_o, total;
+};
+
+WsLayout ws_layout(const Shape& s, int64_t len, int32_t f) {
+  WsLayout w{};
+  const int64_t M = blocks_of(len);
+  size_t off = kCtrlBytes;
+  w.scores = off;
+  off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(float));
+  w.sel = off;
+  off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(int32_t));
+  // decode rows: B*Hq with units B*H; rectify rows: B*f*Hq with units B*H*f
+  const int64_t dec = static_cast<int64_t>(s.B) * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H);
+  const int64_t fr = f > 0 ? f : 1;
+  const int64_t rec = static_cast<int64_t>(s.B) * fr * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H * fr);
+  const int64_t rows = dec > rec ? dec : rec;
+  w.part_ml = off;
+  off = align_up(off + static_cast<size_t>(rows) * 2 * sizeof(float));
+  w.part_o = off;
+  off = align_up(off + static_cast<size_t>(rows) * s.D * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? RESA_OK : RESA_ERR_CUDA; }
+
+// split-KV attention over `R` query rows + merge
+int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int32_t* sel, int n_sel,
+                  float scale, const void* k, const void* v, void* out, float* lse, uint8_t* ws,
+                  const WsLayout& w, int num_sms, cudaStream_t st) {
+  const int64_t min_blocks = sel ? n_sel : blocks_of(len0);
+  const int S = splits_for(s.B * s.H * R, min_blocks, num_sms, s);
+  AttnArgs a{};
+  a.q = q; a.R = R; a.len0 = len0; a.sel = sel; a.n_sel = n_sel; a.S = S; a.scale = scale;
+  a.part_o = reinterpret_cast<float*>(ws + w.part_o);
+  a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  a.ctrl = reinterpret_cast<Ctrl*>(ws);
+  a.k = k; a.v = v;
+  CUtensorMap tk, tv;
+  if (s.bf16) {
+    if (!make_cache_map(&tk, k, s) || !make_cache_map(&tv, v, s)) return RESA_ERR_CUDA;
+    a.tm_k = &tk;
+    a.tm_v = &tv;
+  }
+  cudaError_t e = launch_attend(s, a, st);
+  if (e != cudaSuccess) return RESA_ERR_CUDA;
+  return cuda_status(launch_merge(s, R, S, a.part_o, a.part_ml, out, lse, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t resa_num_selected(int64_t len, int32_t block_size, double r, int32_t n_min) {
+  if (len < 1 || block_size != 16 || !(r > 0.0 && r <= 1.0) || n_min < 1) return RESA_ERR_INVALID_ARG;
+  const int64_t M = blocks_of(len);
+  int64_t n = static_cast<int64_t>(std::ceil(static_cast<double>(M) * r - 1e-9));
+  if (n < n_min) n = n_min;
+  if (n > M) n = M;
+  return static_cast<int32_t>(n);
+}
+
+size_t resa_workspace_bytes(const resa_dims* dims, int64_t len, int32_t f) {
+  Shape s;
+  if (check_dims(dims, &s) != RESA_OK || len < 1 || f < 0) return 0;
+  return ws_layout(s, len, f).total;
+}
+
+int resa_build_desc(const resa_dims* dims, const void* k_cache, int64_t len, void* desc,
+                    void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != RESA_OK) return rc;
+  if (!k_cache || !desc || !aligned16(k_cache) || !aligned16(desc) || len < 1) return RESA_ERR_INVALID_ARG;
+  if (len > s.L_max) return RESA_ERR_CAPACITY;
+  return cuda_status(launch_build_desc(s, k_cache, desc, len, static_cast<cudaStream_t>(stream)));
+}
+
+static int check_decode_common(const resa_dims* dims, Shape* s, const void* q, const void* k_new,
+                               const void* v_new, const void* k_cache, const void* v_cache,
+                               int64_t len, const void* out, const void* workspace,
+                               size_t workspace_bytes, int32_t f_for_ws) {
+  int rc = check_dims(dims, s);
+  if (rc != RESA_OK) return rc;
+  if (!q || !k_cache || !v_cache || !out || !workspace) return RESA_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return RESA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (k_new && (!aligned16(k_new) || !aligned16(v_new))) ||
+      (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return RESA_ERR_INVALID_ARG;
+  if (len < 1) return RESA_ERR_INVALID_ARG;
+  if (len > s->L_max) return RESA_ERR_CAPACITY;
+  if (workspace_bytes < ws_layout(*s, len, f_for_ws).total) return RESA_ERR_WORKSPACE;
+  return RESA_OK;
+}
+
+int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
+                       const void* v_new, void* k_cache, void* v_cache, void* desc,
+                       int64_t len, double r, int32_t n_min, float softmax_scale, void* out,
+                       float* lse, int32_t* sel, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  Shape s;
+  int rc = check_decode_common(dims, &s, q, k_new, v_new, k_cache, v_cache, len, out, workspace,
+                               workspace_bytes, 0);
+  if (rc != RESA_OK) return rc;
+  if (!desc || !aligned16(desc)) return RESA_ERR_INVALID_ARG;
+  if (!(r > 0.0 && r <= 1.0) || n_min < 1 || !std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
+  const int num_sms = device_sms();
+  if (num_sms <= 0) return RESA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int M = static_cast<int>(blocks_of(len));
+  const int n = resa_num_selected(len, 16, r, n_min);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout w = ws_layout(s, len, 0);
+  float* scores = reinterpret_cast<float*>(ws + w.scores);
+  int32_t* selp = sel ? sel : reinterpret_cast<int32_t*>(ws + w.sel);
+
+  cudaError_t e = launch_score(s, q, desc, scores, k_new, v_new, k_cache, v_cache, desc, len,
+                               num_sms, st);
+  if (e != cudaSuccess) return RESA_ERR_CUDA;
+  e = launch_select(s, scores, selp, M, n, st);
+  if (e != cudaSuccess) return RESA_ERR_CUDA;
+  return run_attention(s, q, 1, len, selp, n, softmax_scale, k_cache, v_cache, out, lse, ws, w,
+                       num_sms, st);
+}
+
+int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
+                      const void* v_new, void* k_cache, void* v_cache, void* desc, int64_t len,
+                      float softmax_scale, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_decode_common(dims, &s, q, k_new, v_new, k_cache, v_cache, len, out, workspace,
+                               workspace_bytes, 0);
+  if (rc != RESA_OK) return rc;
+  if (desc && !aligned16(desc)) return RESA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
+  const int num_sms = device_sms();
+  if (num_sms <= 0) return RESA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout w = ws_layout(s, len, 0);
+  if (k_new) {
+    cudaError_t e = launch_append(s, k_new, v_new, k_cache, v_cache, desc, len, st);
+    if (e != cudaSuccess) return RESA_ERR_CUDA;
+  }
+  return run_attention(s, q, 1, len, nullptr, 0, softmax_scale, k_cache, v_cache, out, lse, ws, w,
+                       num_sms, st);
+}
+
+int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
+                 void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
+                 float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  Shape s;
+  int rc = check_dims(dims, &s);
+  if (rc != RESA_OK) return rc;
+  if (f < 1) return RESA_ERR_INVALID_ARG;
+  rc = check_decode_common(dims, &s, q_f, k_f, v_f, k_cache, v_cache, len, out_f, workspace,
+                               workspace_bytes, f);
+  if (rc != RESA_OK) return rc;
+  if (!k_f || !desc || !aligned16(desc)) return RESA_ERR_INVALID_ARG;
+  if (f > len || !std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
+  const int num_sms = device_sms();
+  if (num_sms <= 0) return RESA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout w = ws_layout(s, len, f);
+  cudaError_t e = launch_rectify_write(s, k_f, v_f, k_cache, v_cache, desc, len, f, st);
+  if (e != cudaSuccess) return RESA_ERR_CUDA;
+  return run_attention(s, q_f, f, len - f + 1, nullptr, 0, softmax_scale, k_cache, v_cache, out_f,
+                       nullptr, ws, w, num_sms, st);
+}
+
+int resa_workspace_status(void* workspace, void* stream) {
+  if (!workspace) return RESA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RESA_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpy(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return RESA_ERR_CUDA;
+  if (err != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return RESA_ERR_CUDA;
+    return RESA_ERR_TIMEOUT;
+  }
+  return RESA_OK;
+}
+
+const char* resa_status_string(int status) {
+  switch (status) {
+    case RESA_OK: return "ok";
+    case RESA_ERR_INVALID_ARG: return "invalid argument";
+    case RESA_ERR_UNSUPPORTED: return "unsupported shape (head_dim 64/128, group <= 8, block 16)";
+    case RESA_ERR_CAPACITY: return "len exceeds cache capacity";
+    case RESA_ERR_WORKSPACE: return "workspace too small";
+    case RESA_ERR_CUDA: return "CUDA error";
+    case RESA_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

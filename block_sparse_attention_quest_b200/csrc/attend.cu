@@ -1,0 +1,485 @@
+// Split-KV block-sparse attention and the log-sum-exp merge of the splits.
+//
+// "Rectified Sparse Attention" (pith.science review), section "What carries
+// the argument": all heads of a GQA group read the same selected key blocks;
+// Eq. 2 (minor comment 3) masks token k through its block floor(k / b). The
+// split/merge schedule follows Flash-Decoding (reference list of the same
+// page): each CTA reduces a contiguous slice of the group's block list to an
+// unnormalised (max, sum, accumulator) triple and a second kernel merges them.
+//
+// One CTA serves every query head of one KV group for one query row and one
+// slice of blocks, so a gathered K/V block is fetched from HBM once and used
+// by all G heads.
+//
+// bf16 path: each warp owns a private ring of STAGES tiles; a tile is the K
+// and V rows of one 16-token block, brought in by 2-D TMA tensor copies with
+// 128-byte swizzle (conflict-free ldmatrix). The per-block products
+// S^T = K q^T (16 tokens x 8 head columns, k = head_dim) and O^T += V^T P^T
+// run on warp-level mma.sync; the softmax is the usual online update in
+// float32 and the probabilities enter the second product as bf16.
+//
+// fp32 path: the same schedule on CUDA cores with plain loads (no tensor
+// cores: fp32 inputs must keep fp32 products).
+#include "launch.h"
+
+namespace resa {
+
+struct AttnK {
+  const void* q;
+  const int32_t* sel;
+  float* part_o;
+  float* part_ml;
+  Ctrl* ctrl;
+  const void* k;
+  const void* v;
+  int64_t len0;
+  int64_t L_max;
+  int R, Hq, H, G, n_sel, S;
+  float scale_log2;
+};
+
+__device__ __forceinline__ void split_range(const AttnK& a, int s, int64_t len_r, int& i0,
+                                            int& i1) {
+  const int n = a.sel ? a.n_sel : static_cast<int>((len_r + kBlock - 1) / kBlock);
+  i0 = static_cast<int>(static_cast<int64_t>(s) * n / a.S);
+  i1 = static_cast<int>(static_cast<int64_t>(s + 1) * n / a.S);
+}
+
+// Merge the per-warp (m, l, O) of one CTA through shared memory and write the
+// CTA's partial. sm must hold NW * 8 * (D + 2) floats.
+template <int D, int NW>
+__device__ __forceinline__ void cta_merge_write(const AttnK& a, float* sm, int br, int g,
+                                                int s_idx) {
+  float* sm_o = sm;                       // [NW][8][D]
+  float* sm_m = sm + NW * 8 * D;          // [NW][8]
+  float* sm_l = sm_m + NW * 8;            // [NW][8]
+  for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
+    const int h = idx / D, ch = idx % D;
+    float mstar = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mstar = fmaxf(mstar, sm_m[w * 8 + h]);
+    float o = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float sc = mstar == -INFINITY ? 0.f : exp2f(sm_m[w * 8 + h] - mstar);
+      o = fmaf(sc, sm_o[(w * 8 + h) * D + ch], o);
+      l = fmaf(sc, sm_l[w * 8 + h], l);
+    }
+    const int64_t row = (static_cast<int64_t>(br) * a.Hq + g * a.G + h) * a.S + s_idx;
+    a.part_o[row * D + ch] = o;
+    if (ch == 0) {
+      a.part_ml[row * 2] = mstar;
+      a.part_ml[row * 2 + 1] = l;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------- bf16
+template <int D, int NW, int STAGES>
+struct Bf16Cfg {
+  static constexpr int kHalf = 16 * 64 * 2;            // one 16 x 64 bf16 box (2 KB)
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTile = 2 * kHalves * kHalf;    // K and V of one block
+  static constexpr int kSmem = NW * STAGES * kTile + 1024;
+};
+
+template <int D, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                              const __grid_constant__ CUtensorMap tmV,
+                                                              AttnK a) {
+  using Cfg = Bf16Cfg<D, NW, STAGES>;
+  constexpr int KT = D / 16;                 // k-steps of the QK product, m-tiles of PV
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[NW][STAGES];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+
+  const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
+  const int b = br / a.R, r = br % a.R;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t len_r = a.len0 + r;
+  int i0, i1;
+  split_range(a, s_idx, len_r, i0, i1);
+  const int span = i1 - i0;
+  const int my_count = span > warp ? (span - warp + NW - 1) / NW : 0;
+  const int32_t* selp = a.sel ? a.sel + (static_cast<int64_t>(b) * a.H + g) * a.n_sel : nullptr;
+  const int64_t row_base = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
+
+  if (lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bars[warp][st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  auto block_of = [&](int k) -> int {
+    const int i = i0 + warp + k * NW;
+    return selp ? selp[i] : i;
+  };
+  auto issue = [&](int k) {
+    const int st = k % STAGES;
+    const int j = block_of(k);
+    const int y = static_cast<int>(row_base + static_cast<int64_t>(j) * kBlock);
+    uint8_t* t = tiles + (warp * STAGES + st) * Cfg::kTile;
+    mbar_arrive_expect_tx(&bars[warp][st], Cfg::kTile);
+#pragma unroll
+    for (int hf = 0; hf < Cfg::kHalves; ++hf) {
+      tma_load_2d(t + hf * Cfg::kHalf, &tmK, hf * 64, y, &bars[warp][st]);
+      tma_load_2d(t + (Cfg::kHalves + hf) * Cfg::kHalf, &tmV, hf * 64, y, &bars[warp][st]);
+    }
+  };
+  if (lane == 0) {
+    for (int k = 0; k < my_count && k < STAGES; ++k) issue(k);
+  }
+
+  // q^T as the B operand: lane (gq = lane / 4, c = lane % 4) holds head gq,
+  // channels kk*16 + 2c, +1 (b0) and kk*16 + 8 + 2c, +1 (b1)
+  const int gq = lane >> 2, cq = lane & 3;
+  uint32_t qb[KT][2];
+  {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) +
+                                (static_cast<int64_t>(br) * a.Hq + g * a.G + gq) * D;
+#pragma unroll
+    for (int kk = 0; kk < KT; ++kk) {
+      if (gq < a.G) {
+        qb[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * cq);
+        qb[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * cq);
+      } else {
+        qb[kk][0] = 0u;
+        qb[kk][1] = 0u;
+      }
+    }
+  }
+
+  float o[KT][4];
+#pragma unroll
+  for (int mt = 0; mt < KT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const float sl2 = a.scale_log2;
+  // ldmatrix row/chunk owned by this lane
+  const int kq_row = (lane & 7) + (((lane >> 3) & 1) << 3);   // K (non-trans) row
+  const int kq_chk = lane >> 4;                                // + 2*kk
+  const int vt_row = (lane & 7) + ((lane >> 4) << 3);          // V (trans) row
+  const int vt_chk = (lane >> 3) & 1;                          // + 2*mt
+  bool ok = true;
+  int k = 0;
+  for (; k < my_count; ++k) {
+    const int st = k % STAGES;
+    const bool arrived = mbar_wait_bounded(&bars[warp][st], (k / STAGES) & 1, a.ctrl);
+    if (!__all_sync(0xffffffffu, arrived)) { ok = false; break; }
+    const int j = block_of(k);
+    const uint32_t tbase = smem_u32(tiles + (warp * STAGES + st) * Cfg::kTile);
+    const uint32_t vbase = tbase + Cfg::kHalves * Cfg::kHalf;
+
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < KT; ++kk) {
+      const int chunk = 2 * kk + kq_chk;
+      const uint32_t addr = tbase + (chunk >> 3) * Cfg::kHalf + kq_row * 128 +
+                            (((chunk & 7) ^ (kq_row & 7)) << 4);
+      uint32_t af[4];
+      ldmatrix_x4(af, addr);
+      mma_bf16_16816(sacc, af, qb[kk][0], qb[kk][1]);
+    }
+    // sacc: (token gq, head 2cq), (gq, 2cq+1), (gq+8, 2cq), (gq+8, 2cq+1)
+    const int64_t t_lo = static_cast<int64_t>(j) * kBlock + gq;
+    float s0 = sacc[0] * sl2, s1 = sacc[1] * sl2, s2 = sacc[2] * sl2, s3 = sacc[3] * sl2;
+    if (t_lo >= len_r) { s0 = -INFINITY; s1 = -INFINITY; }
+    if (t_lo + 8 >= len_r) { s2 = -INFINITY; s3 = -INFINITY; }
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+    mx0 = warp_max_xor(mx0, 16, 4);
+    mx1 = warp_max_xor(mx1, 16, 4);
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+    const float p0 = exp2f(s0 - mn0), p2 = exp2f(s2 - mn0);
+    const float p1 = exp2f(s1 - mn1), p3 = exp2f(s3 - mn1);
+    l0 = fmaf(l0, al0, p0 + p2);
+    l1 = fmaf(l1, al1, p1 + p3);
+    m0 = mn0;
+    m1 = mn1;
+#pragma unroll
+    for (int mt = 0; mt < KT; ++mt) {
+      o[mt][0] *= al0; o[mt][2] *= al0;
+      o[mt][1] *= al1; o[mt][3] *= al1;
+    }
+    // P^T as the B operand of O^T += V^T P^T
+    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+#pragma unroll
+    for (int mt = 0; mt < KT; ++mt) {
+      const int chunk = 2 * mt + vt_chk;
+      const uint32_t addr = vbase + (chunk >> 3) * Cfg::kHalf + vt_row * 128 +
+                            (((chunk & 7) ^ (vt_row & 7)) << 4);
+      uint32_t af[4];
+      ldmatrix_x4_trans(af, addr);
+      mma_bf16_16816(o[mt], af, pb0, pb1);
+    }
+    __syncwarp();
+    if (lane == 0 && k + STAGES < my_count) {
+      fence_proxy_async_smem();
+      issue(k + STAGES);
+    }
+  }
+  if (!ok) {
+    // drain the copies this warp still has in flight (bounded), then leave
+    // without writing a partial; the host sees the error flag
+    for (int kk = k; kk < my_count && kk < k + STAGES; ++kk)
+      mbar_wait_bounded(&bars[warp][kk % STAGES], (kk / STAGES) & 1, a.ctrl);
+  }
+  const bool cta_ok = __syncthreads_and(ok);
+  if (!cta_ok) return;
+
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 4);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 8);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 16);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 4);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 8);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 16);
+
+  float* sm = reinterpret_cast<float*>(tiles);
+  float* sm_o = sm;
+  float* sm_m = sm + NW * 8 * D;
+  float* sm_l = sm_m + NW * 8;
+  const int h0 = 2 * cq, h1 = 2 * cq + 1;
+  if (gq == 0) {
+    sm_m[warp * 8 + h0] = m0; sm_l[warp * 8 + h0] = l0;
+    sm_m[warp * 8 + h1] = m1; sm_l[warp * 8 + h1] = l1;
+  }
+#pragma unroll
+  for (int mt = 0; mt < KT; ++mt) {
+    const int ch = mt * 16 + gq;
+    sm_o[(warp * 8 + h0) * D + ch] = o[mt][0];
+    sm_o[(warp * 8 + h1) * D + ch] = o[mt][1];
+    sm_o[(warp * 8 + h0) * D + ch + 8] = o[mt][2];
+    sm_o[(warp * 8 + h1) * D + ch + 8] = o[mt][3];
+  }
+  __syncthreads();
+  cta_merge_write<D, NW>(a, sm, br, g, s_idx);
+}
+
+// ---------------------------------------------------------------------- fp32
+template <int D, int NW>
+__global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
+  constexpr int P = D + 1;                    // padded row (conflict-free column reads)
+  constexpr int CPL = D / 32;                 // output channels per lane
+  extern __shared__ float smf[];
+  float* sq = smf;                            // [8][D]
+  float* tiles = smf + 8 * D;                 // [NW][2][16][P]
+  const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
+  const int b = br / a.R, r = br % a.R;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t len_r = a.len0 + r;
+  const float* qrow = static_cast<const float*>(a.q) + (static_cast<int64_t>(br) * a.Hq + g * a.G) * D;
+  for (int i = threadIdx.x; i < a.G * D; i += NW * 32) sq[i] = qrow[i];
+  __syncthreads();
+  int i0, i1;
+  split_range(a, s_idx, len_r, i0, i1);
+  const int32_t* selp = a.sel ? a.sel + (static_cast<int64_t>(b) * a.H + g) * a.n_sel : nullptr;
+  const int64_t row_base = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
+  const float* kc = static_cast<const float*>(a.k);
+  const float* vc = static_cast<const float*>(a.v);
+  float* Ks = tiles + warp * 2 * 16 * P;
+  float* Vs = Ks + 16 * P;
+
+  float m[8], l[8], acc[8][CPL];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) acc[h][i] = 0.f;
+  }
+  const int t = lane & 15, half = lane >> 4;
+  for (int i = i0 + warp; i < i1; i += NW) {
+    const int j = selp ? selp[i] : i;
+    const float* kb = kc + (row_base + static_cast<int64_t>(j) * kBlock) * D;
+    const float* vb = vc + (row_base + static_cast<int64_t>(j) * kBlock) * D;
+    __syncwarp();
+    for (int e = lane; e < 16 * D / 4; e += 32) {
+      const int row = e / (D / 4), c4 = (e % (D / 4)) * 4;
+      const float4 kv = *reinterpret_cast<const float4*>(kb + row * D + c4);
+      const float4 vv = *reinterpret_cast<const float4*>(vb + row * D + c4);
+      Ks[row * P + c4] = kv.x; Ks[row * P + c4 + 1] = kv.y;
+      Ks[row * P + c4 + 2] = kv.z; Ks[row * P + c4 + 3] = kv.w;
+      Vs[row * P + c4] = vv.x; Vs[row * P + c4 + 1] = vv.y;
+      Vs[row * P + c4 + 2] = vv.z; Vs[row * P + c4 + 3] = vv.w;
+    }
+    __syncwarp();
+    const bool valid = static_cast<int64_t>(j) * kBlock + t < len_r;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h < a.G) {
+        float part = 0.f;
+#pragma unroll 8
+        for (int c = half * (D / 2); c < (half + 1) * (D / 2); ++c)
+          part = fmaf(sq[h * D + c], Ks[t * P + c], part);
+        part += __shfl_xor_sync(0xffffffffu, part, 16);
+        const float z = valid ? part * a.scale_log2 : -INFINITY;
+        float mx = z;
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float mn = fmaxf(m[h], mx);
+        const float al = exp2f(m[h] - mn);
+        const float p = exp2f(z - mn);
+        float ps = p;
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        l[h] = fmaf(l[h], al, ps);
+        m[h] = mn;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) acc[h][i] *= al;
+#pragma unroll
+        for (int tt = 0; tt < 16; ++tt) {
+          const float pt = __shfl_sync(0xffffffffu, p, tt);
+#pragma unroll
+          for (int i = 0; i < CPL; ++i) acc[h][i] = fmaf(pt, Vs[tt * P + lane + 32 * i], acc[h][i]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  float* sm = tiles;                       // reuse: needs NW*8*(D+2) floats
+  float* sm_o = sm;
+  float* sm_m = sm + NW * 8 * D;
+  float* sm_l = sm_m + NW * 8;
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    if (h < a.G) {
+      if (lane == 0) { sm_m[warp * 8 + h] = m[h]; sm_l[warp * 8 + h] = l[h]; }
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) sm_o[(warp * 8 + h) * D + lane + 32 * i] = acc[h][i];
+    }
+  }
+  __syncthreads();
+  cta_merge_write<D, NW>(a, sm, br, g, s_idx);
+}
+
+// ---------------------------------------------------------------------- merge
+template <typename T, int D>
+__global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ part_o,
+                                                    const float* __restrict__ part_ml,
+                                                    T* __restrict__ out, float* __restrict__ lse,
+                                                    int Hq, int S) {
+  constexpr int CPL = D / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = blockIdx.x * 4 + warp;
+  if (h >= Hq) return;
+  const int64_t row = static_cast<int64_t>(blockIdx.y) * Hq + h;
+  const float* ml = part_ml + row * S * 2;
+  float ms[2], ls[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int s = lane + 32 * q;
+    ms[q] = s < S ? ml[2 * s] : -INFINITY;
+    ls[q] = s < S ? ml[2 * s + 1] : 0.f;
+  }
+  float mstar = fmaxf(ms[0], ms[1]);
+  mstar = warp_max_xor(mstar, 16, 1);
+  float w[2], lsum = 0.f;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    w[q] = ms[q] == -INFINITY ? 0.f : exp2f(ms[q] - mstar);
+    lsum = fmaf(w[q], ls[q], lsum);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  float acc[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
+  const float* po = part_o + row * S * D + lane * CPL;
+  for (int s = 0; s < S; ++s) {
+    const float ws = __shfl_sync(0xffffffffu, w[s >> 5], s & 31);
+    if (CPL == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(s) * D);
+      acc[0] = fmaf(ws, x.x, acc[0]);
+      acc[1] = fmaf(ws, x.y, acc[1]);
+      acc[2] = fmaf(ws, x.z, acc[2]);
+      acc[3] = fmaf(ws, x.w, acc[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) acc[i] = fmaf(ws, po[static_cast<int64_t>(s) * D + i], acc[i]);
+    }
+  }
+  const float inv = 1.f / lsum;
+  T* orow = out + row * D + lane * CPL;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) orow[i] = Dt<T>::from_f(acc[i] * inv);
+  if (lse != nullptr && lane == 0) lse[row] = (mstar + log2f(lsum)) * 0.69314718055994531f;
+}
+
+// ---------------------------------------------------------------------- launch
+constexpr int kNW = 4;
+constexpr int kStages = 3;
+
+template <int D>
+static cudaError_t attend_bf16_t(const Shape& s, const AttnK& k, const AttnArgs& a,
+                                 cudaStream_t st) {
+  using Cfg = Bf16Cfg<D, kNW, kStages>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<D, kNW, kStages>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(a.S, s.H, s.B * a.R);
+  attend_bf16_kernel<D, kNW, kStages><<<grid, kNW * 32, Cfg::kSmem, st>>>(*a.tm_k, *a.tm_v, k);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t attend_f32_t(const Shape& s, const AttnK& k, const AttnArgs& a,
+                                cudaStream_t st) {
+  const size_t tiles = static_cast<size_t>(kNW) * 2 * 16 * (D + 1);
+  const size_t merge = static_cast<size_t>(kNW) * 8 * (D + 2);
+  const size_t smem = (8 * D + (tiles > merge ? tiles : merge)) * sizeof(float);
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attend_f32_kernel<D, kNW>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(a.S, s.H, s.B * a.R);
+  attend_f32_kernel<D, kNW><<<grid, kNW * 32, smem, st>>>(k);
+  return cudaGetLastError();
+}
+
+int attend_ctas_per_sm(const Shape& s) { return s.bf16 ? 2 : 4; }
+
+cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st) {
+  AttnK k{};
+  k.q = a.q; k.sel = a.sel; k.part_o = a.part_o; k.part_ml = a.part_ml; k.ctrl = a.ctrl;
+  k.k = a.k; k.v = a.v; k.len0 = a.len0; k.L_max = s.L_max; k.R = a.R; k.Hq = s.Hq; k.H = s.H;
+  k.G = s.G; k.n_sel = a.n_sel; k.S = a.S;
+  k.scale_log2 = a.scale * 1.4426950408889634f;
+  if (s.bf16) return s.D == 128 ? attend_bf16_t<128>(s, k, a, st) : attend_bf16_t<64>(s, k, a, st);
+  return s.D == 128 ? attend_f32_t<128>(s, k, a, st) : attend_f32_t<64>(s, k, a, st);
+}
+
+cudaError_t launch_merge(const Shape& s, int R, int S, const float* part_o, const float* part_ml,
+                         void* out, float* lse, cudaStream_t st) {
+  dim3 grid((s.Hq + 3) / 4, s.B * R);
+  if (s.bf16) {
+    using T = __nv_bfloat16;
+    if (s.D == 128)
+      merge_kernel<T, 128><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<T*>(out), lse, s.Hq, S);
+    else
+      merge_kernel<T, 64><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<T*>(out), lse, s.Hq, S);
+  } else {
+    if (s.D == 128)
+      merge_kernel<float, 128><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<float*>(out), lse, s.Hq, S);
+    else
+      merge_kernel<float, 64><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<float*>(out), lse, s.Hq, S);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace resa

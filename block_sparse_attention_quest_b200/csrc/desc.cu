@@ -1,0 +1,188 @@
+// Quest block descriptors: full build, incremental append, and the refresh
+// after a rectification.
+//
+// "Rectified Sparse Attention" (pith.science review), section "What carries
+// the argument": blocks are ranked through Quest-style per-channel min/max
+// block descriptors; rectification replaces KV entries and updates the block
+// statistics. Block size b = 16 ("Assumptions & free parameters").
+//
+// All three kernels are bound by HBM traffic of the keys they read; the
+// min/max of bf16 values is exact in float and converts back exactly.
+#include "launch.h"
+
+namespace resa {
+
+// One warp per (b, h, block). Lane `lane` owns 16-byte chunk lane % CPR of a
+// row and rows lane / CPR, lane / CPR + TPP, ...; lanes that own the same
+// chunk are then combined with xor-shuffles.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) build_desc_kernel(const T* __restrict__ k,
+                                                         T* __restrict__ desc, int64_t L_max,
+                                                         int Mmax, int M, int64_t len,
+                                                         int64_t total) {
+  constexpr int CH = Chunk<T>::N;
+  constexpr int CPR = D / CH;                 // 16-byte chunks per token row
+  constexpr int TPP = 32 / CPR;               // rows covered by one warp-wide load
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= total) return;
+  const int64_t bh = wid / M;
+  const int j = static_cast<int>(wid % M);
+  const int valid = static_cast<int>(len - static_cast<int64_t>(j) * kBlock < kBlock ? len - static_cast<int64_t>(j) * kBlock : kBlock);
+  const int chunk = lane % CPR;
+  const int r0 = lane / CPR;
+  const T* base = k + (bh * L_max + static_cast<int64_t>(j) * kBlock) * D + chunk * CH;
+
+  float mn[CH], mx[CH];
+#pragma unroll
+  for (int e = 0; e < CH; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; }
+  uint4 raw[kBlock / TPP];
+#pragma unroll
+  for (int i = 0; i < kBlock / TPP; ++i) {
+    const int t = r0 + i * TPP;
+    raw[i] = t < valid ? ld_stream16(base + static_cast<int64_t>(t) * D) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < kBlock / TPP; ++i) {
+    const int t = r0 + i * TPP;
+    if (t < valid) {
+      float f[CH];
+      Chunk<T>::unpack(raw[i], f);
+#pragma unroll
+      for (int e = 0; e < CH; ++e) { mn[e] = fminf(mn[e], f[e]); mx[e] = fmaxf(mx[e], f[e]); }
+    }
+  }
+#pragma unroll
+  for (int m = CPR; m < 32; m <<= 1) {
+#pragma unroll
+    for (int e = 0; e < CH; ++e) {
+      mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], m));
+      mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], m));
+    }
+  }
+  if (lane < CPR) {
+    T* d = desc + (bh * Mmax + j) * 2 * D + chunk * CH;
+    *reinterpret_cast<uint4*>(d) = Chunk<T>::pack(mn);
+    *reinterpret_cast<uint4*>(d + D) = Chunk<T>::pack(mx);
+  }
+}
+
+// Decode-time append: token len-1 is written to the cache and merged into the
+// descriptor of its block (or opens it). Grid (H, B), D threads.
+template <typename T>
+__global__ void append_kernel(const T* __restrict__ k_new, const T* __restrict__ v_new,
+                              T* __restrict__ k, T* __restrict__ v, T* __restrict__ desc, int H,
+                              int D, int64_t L_max, int Mmax, int64_t len) {
+  const int c = threadIdx.x;
+  const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
+  const int64_t t = len - 1;
+  const T kn = k_new[bh * D + c];
+  k[(bh * L_max + t) * D + c] = kn;
+  v[(bh * L_max + t) * D + c] = v_new[bh * D + c];
+  if (desc) {
+    T* d = desc + (bh * Mmax + t / kBlock) * 2 * D;
+    if (t % kBlock == 0) {
+      d[c] = kn;
+      d[D + c] = kn;
+    } else {
+      const float x = Dt<T>::to_f(kn);
+      d[c] = Dt<T>::from_f(fminf(Dt<T>::to_f(d[c]), x));
+      d[D + c] = Dt<T>::from_f(fmaxf(Dt<T>::to_f(d[D + c]), x));
+    }
+  }
+}
+
+// Rectify write + refresh: grid (blocks touched, H, B), D threads. The CTA of
+// block j writes the new K/V rows of that block (slots >= len - f), then
+// recomputes the block's min/max over all its valid tokens.
+template <typename T>
+__global__ void rectify_write_kernel(const T* __restrict__ k_f, const T* __restrict__ v_f,
+                                     T* __restrict__ k, T* __restrict__ v, T* __restrict__ desc,
+                                     int H, int D, int64_t L_max, int Mmax, int64_t len, int f) {
+  const int c = threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  const int64_t t_first = len - f;
+  const int64_t j = t_first / kBlock + blockIdx.x;
+  const int64_t t0 = j * kBlock;
+  const int64_t t1 = t0 + kBlock < len ? t0 + kBlock : len;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int64_t t = t0; t < t1; ++t) {
+    T kv;
+    if (t >= t_first) {
+      const int64_t i = t - t_first;
+      const int64_t src = ((static_cast<int64_t>(b) * f + i) * H + h) * D + c;
+      kv = k_f[src];
+      k[(bh * L_max + t) * D + c] = kv;
+      v[(bh * L_max + t) * D + c] = v_f[src];
+    } else {
+      kv = k[(bh * L_max + t) * D + c];
+    }
+    const float x = Dt<T>::to_f(kv);
+    mn = fminf(mn, x);
+    mx = fmaxf(mx, x);
+  }
+  T* d = desc + (bh * Mmax + j) * 2 * D;
+  d[c] = Dt<T>::from_f(mn);
+  d[D + c] = Dt<T>::from_f(mx);
+}
+
+template <typename T, int D>
+static cudaError_t build_desc_t(const Shape& s, const void* k, void* desc, int64_t len,
+                                cudaStream_t st) {
+  const int M = static_cast<int>((len + kBlock - 1) / kBlock);
+  const int64_t total = static_cast<int64_t>(s.B) * s.H * M;
+  const int threads = 256;
+  const int64_t grid = (total * 32 + threads - 1) / threads;
+  build_desc_kernel<T, D><<<static_cast<unsigned>(grid), threads, 0, st>>>(
+      static_cast<const T*>(k), static_cast<T*>(desc), s.L_max, s.Mmax, M, len, total);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_desc(const Shape& s, const void* k, void* desc, int64_t len,
+                              cudaStream_t st) {
+  if (s.bf16) {
+    return s.D == 128 ? build_desc_t<__nv_bfloat16, 128>(s, k, desc, len, st)
+                      : build_desc_t<__nv_bfloat16, 64>(s, k, desc, len, st);
+  }
+  return s.D == 128 ? build_desc_t<float, 128>(s, k, desc, len, st)
+                    : build_desc_t<float, 64>(s, k, desc, len, st);
+}
+
+cudaError_t launch_append(const Shape& s, const void* k_new, const void* v_new, void* k, void* v,
+                          void* desc, int64_t len, cudaStream_t st) {
+  dim3 grid(s.H, s.B);
+  if (s.bf16) {
+    using T = __nv_bfloat16;
+    append_kernel<T><<<grid, s.D, 0, st>>>(static_cast<const T*>(k_new),
+                                           static_cast<const T*>(v_new), static_cast<T*>(k),
+                                           static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D,
+                                           s.L_max, s.Mmax, len);
+  } else {
+    append_kernel<float><<<grid, s.D, 0, st>>>(
+        static_cast<const float*>(k_new), static_cast<const float*>(v_new),
+        static_cast<float*>(k), static_cast<float*>(v), static_cast<float*>(desc), s.H, s.D,
+        s.L_max, s.Mmax, len);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_f, void* k, void* v,
+                                 void* desc, int64_t len, int f, cudaStream_t st) {
+  const int64_t j0 = (len - f) / kBlock;
+  const int64_t M = (len + kBlock - 1) / kBlock;
+  dim3 grid(static_cast<unsigned>(M - j0), s.H, s.B);
+  if (s.bf16) {
+    using T = __nv_bfloat16;
+    rectify_write_kernel<T><<<grid, s.D, 0, st>>>(
+        static_cast<const T*>(k_f), static_cast<const T*>(v_f), static_cast<T*>(k),
+        static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f);
+  } else {
+    rectify_write_kernel<float><<<grid, s.D, 0, st>>>(
+        static_cast<const float*>(k_f), static_cast<const float*>(v_f), static_cast<float*>(k),
+        static_cast<float*>(v), static_cast<float*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace resa

@@ -1,0 +1,63 @@
+// Internal launchers of libresa (host side). Every launcher enqueues on
+// `stream` and returns the cudaError_t of the launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace resa {
+
+struct Shape {
+  int B, Hq, H, G, D;
+  int64_t L_max;   // cache capacity (tokens)
+  int Mmax;        // L_max / 16
+  bool bf16;
+};
+
+// descriptors ----------------------------------------------------------------
+cudaError_t launch_build_desc(const Shape& s, const void* k, void* desc, int64_t len,
+                              cudaStream_t st);
+cudaError_t launch_append(const Shape& s, const void* k_new, const void* v_new, void* k, void* v,
+                          void* desc, int64_t len, cudaStream_t st);
+cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_f, void* k, void* v,
+                                 void* desc, int64_t len, int f, cudaStream_t st);
+
+// scoring + selection ----------------------------------------------------------
+// scores: [B][H][M] float; the CTA that owns the last chunk also performs the
+// append of (k_new, v_new) when k_new != nullptr.
+cudaError_t launch_score(const Shape& s, const void* q, const void* desc, float* scores,
+                         const void* k_new, const void* v_new, void* k, void* v, void* desc_w,
+                         int64_t len, int num_sms, cudaStream_t st);
+cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int M, int n,
+                          cudaStream_t st);
+
+// attention ---------------------------------------------------------------------
+struct AttnArgs {
+  const void* q;          // element (b, r, h, c) at ((b*R + r)*Hq + h)*D + c
+  int R;                  // query rows per batch entry
+  int64_t len0;           // row r sees tokens t < len0 + r
+  const int32_t* sel;     // [B][H][n_sel] or nullptr (dense: every block)
+  int n_sel;
+  int S;                  // splits per (b, r, KV head)
+  float scale;            // softmax scale (natural units)
+  float* part_o;          // [B*R*Hq][S][D]
+  float* part_ml;         // [B*R*Hq][S][2]  (max in log2 units, sum)
+  Ctrl* ctrl;
+  const CUtensorMap* tm_k;  // bf16 only (host copies, passed by value to the kernel)
+  const CUtensorMap* tm_v;
+  const void* k;          // cache base pointers (fp32 path)
+  const void* v;
+};
+cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st);
+int attend_ctas_per_sm(const Shape& s);
+
+// out: [B*R][Hq][D] in the cache dtype; lse: [B*R][Hq] or nullptr
+cudaError_t launch_merge(const Shape& s, int R, int S, const float* part_o, const float* part_ml,
+                         void* out, float* lse, cudaStream_t st);
+
+constexpr int kMaxSplits = 64;
+
+}  // namespace resa

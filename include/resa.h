@@ -1,0 +1,165 @@
+/*
+ * resa.h - C ABI of libresa.so, the B200 (sm_100a) implementation of the
+ * attention hot path of Rectified Sparse Attention (ReSA, arXiv 2506.04108).
+ *
+ * Method (pages describing ReSA; "Rectified Sparse Attention", pith.science
+ * review, section "What carries the argument", Eq. 2, Eq. 5, Eq. 6):
+ *   - group block sparse attention (GBSA): keys are cut into blocks of b = 16
+ *     tokens; each block keeps a per-channel min/max descriptor (Quest); every
+ *     GQA group scores all blocks with the pooled Quest bound and all query
+ *     heads of the group attend to the same top-n blocks;
+ *   - n = max(n_min, ceil(M r)) with M the number of blocks and r the active
+ *     block ratio (Eq. 5; the pages' p read as the active ratio), capped at M;
+ *   - the block that holds the newest token is always kept (n_local = 1);
+ *   - dense rectification: every f decode steps the last f tokens are
+ *     re-encoded with dense causal attention, their KV entries replaced and
+ *     the block statistics updated.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *     and 16-byte aligned. The library allocates no memory and keeps no state
+ *     between calls apart from a per-device cache of launch attributes.
+ *   - Layouts (row-major, innermost last):
+ *       k_cache, v_cache  [batch][n_kv_heads][max_len][head_dim]
+ *       desc              [batch][n_kv_heads][max_len/16][2][head_dim]
+ *                         (row 0 = per-channel min, row 1 = max of the valid
+ *                          keys of the block; same dtype as the cache)
+ *       q, out            [batch][n_q_heads][head_dim]
+ *       k_new, v_new      [batch][n_kv_heads][head_dim]
+ *       q_f, out_f        [batch][f][n_q_heads][head_dim]
+ *       k_f, v_f          [batch][f][n_kv_heads][head_dim]
+ *       lse               [batch][n_q_heads]           float32
+ *       sel               [batch][n_kv_heads][n]        int32, ascending
+ *   - Query head h reads KV head h / (n_q_heads / n_kv_heads).
+ *   - `len` is the number of valid tokens in the cache, counting the token a
+ *     decode call appends. All batch rows share one len.
+ *   - q, k, v, desc and out share the dtype in resa_dims.dtype; softmax and
+ *     accumulation are float32.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
+ *     only enqueues work on it and returns; nothing synchronises.
+ *   - `workspace` is caller-provided device scratch of at least
+ *     resa_workspace_bytes() bytes, 256-byte aligned. Its first 256 bytes are
+ *     a control block: zero them once before first use. Calls that share one
+ *     workspace must be ordered on one stream.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid argument returns a negative resa_status and launches nothing.
+ *     A failed launch returns RESA_ERR_CUDA. A device-side wait that gives up
+ *     sets a flag in the workspace control block, read by
+ *     resa_workspace_status().
+ */
+#ifndef RESA_H_
+#define RESA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RESA_API __attribute__((visibility("default")))
+#else
+#define RESA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RESA_OK = 0,
+  RESA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misalignment, len/f/r out of range */
+  RESA_ERR_UNSUPPORTED = -2,  /* head_dim not 64/128, group > 8, block_size != 16 */
+  RESA_ERR_CAPACITY = -3,     /* len > max_len */
+  RESA_ERR_WORKSPACE = -4,    /* workspace smaller than resa_workspace_bytes() */
+  RESA_ERR_CUDA = -5,         /* a CUDA runtime/driver call or launch failed */
+  RESA_ERR_TIMEOUT = -6       /* a device-side wait gave up (flag in the workspace) */
+} resa_status;
+
+typedef enum { RESA_F32 = 0, RESA_BF16 = 1 } resa_dtype;
+
+typedef struct {
+  int32_t batch;       /* B >= 1 */
+  int32_t n_q_heads;   /* H_q, a multiple of n_kv_heads */
+  int32_t n_kv_heads;  /* H_kv >= 1; group G = H_q / H_kv must be <= 8 */
+  int32_t head_dim;    /* d: 64 or 128 */
+  int32_t block_size;  /* b: must be 16 */
+  int32_t dtype;       /* resa_dtype of q, k, v, desc, out */
+  int64_t max_len;     /* cache capacity in tokens, a positive multiple of 16 */
+} resa_dims;
+
+/* Block budget of Eq. 5: M = ceil(len / 16) blocks (the partial block counts),
+ * n = min(M, max(n_min, ceil(M * r))) with ceil(M * r) evaluated in double as
+ * ceil(M * r - 1e-9). Returns n, or a negative resa_status for len < 1,
+ * r not in (0, 1], n_min < 1 or block_size != 16. */
+RESA_API int32_t resa_num_selected(int64_t len, int32_t block_size, double r, int32_t n_min);
+
+/* Workspace bytes that suffice for resa_decode_sparse, resa_decode_dense and
+ * resa_rectify (with this f) at any length up to `len`. Returns 0 for invalid
+ * dims. */
+RESA_API size_t resa_workspace_bytes(const resa_dims* dims, int64_t len, int32_t f);
+
+/* Quest block descriptors of the first `len` tokens (per-block, per-channel
+ * key minimum and maximum; section "What carries the argument"): for every batch
+ * row, KV head and block j < ceil(len/16), desc[..][j][0][c] = min and
+ * desc[..][j][1][c] = max of k_cache[..][t][c] over the valid tokens
+ * t in [16 j, min(16 j + 16, len)). Blocks at or past ceil(len/16) are not
+ * written. */
+RESA_API int resa_build_desc(const resa_dims* dims, const void* k_cache, int64_t len, void* desc,
+                    void* stream);
+
+/* One GBSA decode step (section "What carries the argument"; Eq. 2, Eq. 5):
+ *  1. if k_new != NULL: write k_new/v_new at slot len-1 and merge k_new into
+ *     the descriptor of block (len-1)/16 (set it to (k_new, k_new) when the
+ *     token opens a new block);
+ *  2. per (batch, KV group) and block j < M-1:
+ *     s_j = sum_{h in group} sum_c max(q_hc * min_jc, q_hc * max_jc);
+ *  3. keep block M-1 plus the n-1 best other blocks (ties to the lower index),
+ *     n = resa_num_selected(len, 16, r, n_min); written ascending to `sel`
+ *     when sel != NULL;
+ *  4. every query head attends (softmax(scale * q.k) v) over the tokens of the
+ *     selected blocks that are < len, split across CTAs and merged by
+ *     log-sum-exp (Flash-Decoding);
+ *  5. out = the result in the cache dtype; lse (if not NULL) = natural-log
+ *     log-sum-exp of the scaled logits.
+ * k_new and v_new are both NULL or both set. */
+RESA_API int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
+                       const void* v_new, void* k_cache, void* v_cache, void* desc,
+                       int64_t len, double r, int32_t n_min, float softmax_scale, void* out,
+                       float* lse, int32_t* sel, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Dense decode of the same step: step 1 of resa_decode_sparse (desc may be
+ * NULL, then descriptors are not updated), then attention over every token
+ * < len. This is the r = 1 comparison arm; it skips scoring and selection. */
+RESA_API int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
+                      const void* v_new, void* k_cache, void* v_cache, void* desc, int64_t len,
+                      float softmax_scale, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* Dense rectification (section "What carries the argument": after every f
+ * decode steps the newest f tokens go through one dense causal pass whose K/V
+ * overwrite the ones the sparse steps produced, and the affected block
+ * summaries are refreshed; f = 32 by default, "Assumptions & free
+ * parameters"):
+ *  1. k_cache/v_cache slots [len-f, len) := k_f/v_f;
+ *  2. descriptors of blocks (len-f)/16 .. ceil(len/16)-1 recomputed from the
+ *     full block contents;
+ *  3. out_f[b][i][h] = causal dense attention of q_f[b][i][h], whose position
+ *     is len-f+i, over keys 0 .. len-f+i.
+ * Requires 1 <= f <= len. */
+RESA_API int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
+                 void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
+                 float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error flag of the
+ * workspace control block. Returns RESA_OK, RESA_ERR_TIMEOUT, or
+ * RESA_ERR_CUDA. */
+RESA_API int resa_workspace_status(void* workspace, void* stream);
+
+/* Human-readable name of a resa_status value (static string). */
+RESA_API const char* resa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RESA_H_ */

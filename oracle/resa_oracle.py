@@ -9,17 +9,18 @@ Sources (all from the pages describing Rectified Sparse Attention, arXiv
 2506.04108):
 
 * "Rectified Sparse Attention" (pith.science review), section "What carries
-  the argument": group block sparse attention (GBSA) in which every GQA group
-  pools its queries and picks the same top blocks through Quest-style min/max
-  block descriptors; every f decode steps a dense pass re-encodes the last f
-  tokens, replaces their KV entries and updates the block statistics; the
-  block budget n = max(n_min, ceil(M p)) (Eq. 5).
+  the argument": group block sparse attention (GBSA), in which one KV
+  group's query heads share a single ranking of key blocks built from Quest's
+  per-block, per-channel key minimum and maximum; after every f decode steps
+  one dense causal pass recomputes the newest f tokens, overwrites their
+  cached keys and values and refreshes the summaries of the blocks involved;
+  the block budget n = max(n_min, ceil(M p)) (Eq. 5).
 * same page, "Referee Report", major comment 1: Eq. 5 uses p as the active
   block ratio (read here as the active ratio r); Eq. 6 memory model.
 * same page, minor comment 3: Eq. 2, the token mask follows its block,
   M^{ijk} = M_{ij floor(k/b)}.
 * same page, "Assumptions & free parameters": b = 16, f = 32, n_min = 16,
-  n_local = 1 ("recent blocks always preserved").
+  n_local = 1 (the newest block is always attended).
 * same page, reference list: Flash-Decoding (split-KV decoding; the split is a
   schedule, the oracle computes the unsplit softmax it must equal) and Quest
   (the min/max descriptor bound).
