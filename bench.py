@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Benchmark of the ReSA decode hot path (libresa.so) on B200.
+
+One benchmark step is one rectification period of one token position across
+`--layers` attention layers: f sparse decode steps (append, score, select,
+split-KV attention, merge) on every layer, then one dense rectification of
+the last f tokens on every layer. The layers hold independent KV caches that
+are visited round-robin, so between two visits of a cache more than the L2
+size (126 MB) of other data is read: the inputs are larger than L2 and no
+explicit flush is needed.
+
+metric: ReSA decode-step us (one attention layer, rectify amortised over f)
+with achieved HBM GB/s against roofline at 128K/256K, and rectify us.
+value = step time / (f * layers * n_gpus) in microseconds (lower is better).
+
+With --gpus N > 1 (torchrun) every rank runs an independent replica of the
+workload (the path has no exchange step); timing is the max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOADS = {"32k": 1, "128k": 2, "256k": 3, "64k": 4}
+WORKLOAD_NAMES = {
+    1: "resa_decode_32k_b4_needles", 2: "resa_decode_128k_b1", 3: "resa_decode_256k_b1",
+    4: "resa_decode_64k_b16",
+}
+METRIC = "ReSA decode-step us & achieved HBM GB/s vs roofline at 128K/256K; rectify us"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--r", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = [x.strip() for x in vis.split(",")] if vis else []
+        self.index = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import __graft_entry__
+    __graft_entry__.build()
+    import block_sparse_attention_quest_b200 as resa
+    from workload import config, decode_inputs, make_cache, rectify_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg_idx = WORKLOADS[args.workload]
+    over = {"steps": 64}
+    if args.r is not None:
+        over["r"] = args.r
+    spec = config(cfg_idx, **over)
+    f, L = spec.f, args.layers
+    tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    esize = 2 if spec.dtype == "bf16" else 4
+    B, Hq, H, d = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+
+    def dev_t(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev).to(tdt)
+
+    K, V = make_cache(spec)
+    k0, v0 = dev_t(K), dev_t(V)
+    del K, V
+    layers = []
+    for li in range(L):
+        k = k0 if li == 0 else k0.clone()
+        v = v0 if li == 0 else v0.clone()
+        desc = torch.zeros(B, H, spec.max_blocks, 2, d, dtype=tdt, device=dev)
+        layers.append(dict(k=k, v=v, desc=desc))
+    dims = resa.dims_for(k0, Hq)
+    ws = [resa.alloc_workspace(dims, spec.max_len, f, device=dev) for _ in range(L)]
+
+    # a1: descriptor build after prefill (timed once per layer, outside the
+    # step; a first untimed pass loads the module)
+    for ly in layers:
+        resa.build_desc(ly["k"], spec.len0, ly["desc"], Hq)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for ly in layers:
+        resa.build_desc(ly["k"], spec.len0, ly["desc"], Hq)
+    ev[1].record()
+    torch.cuda.synchronize()
+    build_desc_us = ev[0].elapsed_time(ev[1]) * 1000.0 / L
+
+    # resident per-step inputs: f decode sets, one rectify set
+    dec_in = []
+    for t in range(f):
+        q, kn, vn = decode_inputs(spec, t)
+        dec_in.append((dev_t(q), dev_t(kn), dev_t(vn)))
+    len_start = spec.len0
+    q_f, k_f, v_f = rectify_inputs(spec, 0, len_start + f, f)
+    rect_in = (dev_t(q_f), dev_t(k_f), dev_t(v_f))
+    n_at = {t: resa.num_selected(len_start + t + 1, spec.r, spec.n_min) for t in range(f)}
+    outs = [torch.empty(B, Hq, d, dtype=tdt, device=dev) for _ in range(L)]
+    lses = [torch.empty(B, Hq, dtype=torch.float32, device=dev) for _ in range(L)]
+    sels = [[torch.empty(B, H, n_at[t], dtype=torch.int32, device=dev) for t in range(f)]
+            for _ in range(L)]
+    out_f = [torch.empty(B, f, Hq, d, dtype=tdt, device=dev) for _ in range(L)]
+
+    # One step = f decode positions x L layers, then L rectifications. Every
+    # replay decodes positions len0 .. len0+f-1 again (the same cache slots are
+    # rewritten with the same values), so each replay does identical work.
+    def step(timing=None):
+        for t in range(f):
+            length = len_start + t + 1
+            q, kn, vn = dec_in[t]
+            for li, ly in enumerate(layers):
+                if timing is None:
+                    resa.decode_sparse(q, kn, vn, ly["k"], ly["v"], ly["desc"], length, spec.r,
+                                       spec.n_min, 1.0, outs[li], ws[li], lse=lses[li],
+                                       sel=sels[li][t])
+                else:
+                    e0, e1, e2 = timing["dec"][t][li]
+                    e0.record()
+                    resa.select_blocks(q, kn, vn, ly["k"], ly["v"], ly["desc"], length, spec.r,
+                                       spec.n_min, sels[li][t], ws[li])
+                    e1.record()
+                    resa.attend_blocks(q, ly["k"], ly["v"], length, sels[li][t], 1.0, outs[li],
+                                       ws[li], lse=lses[li])
+                    e2.record()
+        length = len_start + f
+        for li, ly in enumerate(layers):
+            if timing is not None:
+                timing["rect"][li][0].record()
+            resa.rectify(rect_in[0], rect_in[1], rect_in[2], ly["k"], ly["v"], ly["desc"], length,
+                         f, 1.0, out_f[li], ws[li])
+            if timing is not None:
+                timing["rect"][li][1].record()
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    # eager run once (also validates arguments), then capture
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    assert resa.workspace_status(ws[0]) == resa.RESA_OK
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    mk = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+    timing = {"dec": [[(mk(), mk(), mk()) for _ in range(L)] for _ in range(f)],
+              "rect": [(mk(), mk()) for _ in range(L)]}
+    graph_t = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_t, stream=stream):
+        step(timing)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # warm-up
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # timed region: exactly K replays of the step graph
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = t0.elapsed_time(t1)
+    # keep the GPU busy while the sampler catches a few more readings
+    t_end = time.time() + 0.4
+    while time.time() < t_end:
+        graph.replay()
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    step_ms = total_ms / args.steps
+
+    # per-stage breakdown (graph with captured timing events)
+    reps = max(3, min(args.steps, 10))
+    sel_us, att_us, rect_us = [], [], []
+    for _ in range(reps):
+        graph_t.replay()
+        torch.cuda.synchronize()
+        for t in range(f):
+            for li in range(L):
+                e0, e1, e2 = timing["dec"][t][li]
+                sel_us.append(e0.elapsed_time(e1) * 1000.0)
+                att_us.append(e1.elapsed_time(e2) * 1000.0)
+        for li in range(L):
+            a, b = timing["rect"][li]
+            rect_us.append(a.elapsed_time(b) * 1000.0)
+
+    # end-to-end through the public API with host buffers (eager calls)
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt)
+        if dist is not None:
+            tt = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(tt.item())
+
+    assert resa.workspace_status(ws[0]) == resa.RESA_OK
+    # bytes of the algorithm (descriptors + selected K/V + Q/O)
+    n_mid = n_at[f // 2]
+    len_mid = len_start + f // 2 + 1
+    M_mid = (len_mid + 15) // 16
+    qo = 2 * B * Hq * d * esize
+    desc_bytes = B * H * M_mid * 2 * d * esize
+    sel_kv = B * H * n_mid * 16 * 2 * d * esize
+    attend_bytes = sel_kv + qo + B * H * n_mid * 4
+    decode_bytes = desc_bytes + sel_kv + qo
+    rect_len = len_start + f
+    rect_bytes = B * H * rect_len * 2 * d * esize + 2 * B * f * Hq * d * esize + 2 * B * f * H * d * esize
+    rect_flops = 4.0 * B * Hq * d * (f * rect_len - f * (f - 1) / 2)
+
+    hbm_peak, tf_peak, peak_kind = peaks()
+    sel_med = statistics.median(sel_us)
+    att_med = statistics.median(att_us)
+    rect_med = statistics.median(rect_us)
+    decode_med = statistics.median([a + b for a, b in zip(sel_us, att_us)])
+    att_gbs = attend_bytes / (att_med * 1e-6) / 1e9
+    us_per_decode = step_ms * 1000.0 / (f * L) / world
+    tokens_per_s = B * f * L * world / (step_ms * 1e-3) / L
+    launches_per_step = f * L * 3 + L * 2
+    res = {
+        "metric": METRIC,
+        "value": round(us_per_decode, 3),
+        "unit": "us",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": spec.dtype,
+        "data": "synthetic (seeded N(0,1) + block means; no dataset, no weights)",
+        "config": {
+            "workload": WORKLOAD_NAMES[cfg_idx], "batch": B, "context": spec.len0,
+            "q_heads": Hq, "kv_heads": H, "head_dim": d, "block": 16, "r": spec.r,
+            "n_min": spec.n_min, "f": f, "layers": L,
+            "step": f"{f} sparse decode steps x {L} layers + {L} rectifications",
+            "l2": f"inputs larger than L2: {L} independent layer caches visited round-robin",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "timing": "CUDA graph replay, CUDA events on the launching stream",
+        },
+        "decode_us": round(decode_med, 3),
+        "decode_select_us": round(sel_med, 3),
+        "decode_attend_us": round(att_med, 3),
+        "decode_hbm_gbs": round(decode_bytes / (decode_med * 1e-6) / 1e9, 1),
+        "decode_bytes": decode_bytes,
+        "decode_frac_of_measured_hbm": round(decode_bytes / (decode_med * 1e-6) / 1e9 / hbm_peak, 4),
+        "rectify_us": round(rect_med, 3),
+        "rectify_amortised_us_per_token": round(rect_med / f, 3),
+        "rectify_hbm_gbs": round(rect_bytes / (rect_med * 1e-6) / 1e9, 1),
+        "rectify_tflops": round(rect_flops / (rect_med * 1e-6) / 1e12, 2),
+        "build_desc_us": round(build_desc_us, 2),
+        "tokens_per_s": round(tokens_per_s, 1),
+        "roofline": {
+            "kernel": "attend_bf16_kernel (split-KV attention with the LSE merge in its last CTA)",
+            "bound": "hbm", "achieved": round(att_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(att_gbs / hbm_peak, 4), "traffic": None,
+            "peak_kind": f"{peak_kind} copy bandwidth",
+            "bytes_per_launch": attend_bytes,
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        res["e2e"] = {"value": round(e2e["ms_per_step"] * 1000.0 / (f * L) / world, 3),
+                      "unit": "us", "h2d_bytes_per_step": e2e["h2d"],
+                      "d2h_bytes_per_step": e2e["d2h"]}
+    return res, spec
+
+
+def run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt):
+    """The same step through the public calls, with every step's inputs copied
+    from pinned host memory and every output copied back, inside the timed
+    region."""
+    import torch
+    f, L = spec.f, len(layers)
+    B, Hq, H, d = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+    h_dec = [tuple(x.cpu().pin_memory() for x in s) for s in dec_in]
+    h_rect = tuple(x.cpu().pin_memory() for x in rect_in)
+    d_dec = [tuple(torch.empty_like(x) for x in s) for s in dec_in]
+    d_rect = tuple(torch.empty_like(x) for x in rect_in)
+    out = torch.empty(B, Hq, d, dtype=tdt, device=dev)
+    out_f = torch.empty(B, f, Hq, d, dtype=tdt, device=dev)
+    h_out = torch.empty(L, f, B, Hq, d, dtype=tdt).pin_memory()
+    h_out_f = torch.empty(L, B, f, Hq, d, dtype=tdt).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for s in h_dec for x in s) * L + \
+        sum(x.numel() * x.element_size() for x in h_rect) * L
+    d2h = h_out.numel() * h_out.element_size() + h_out_f.numel() * h_out_f.element_size()
+
+    def step():
+        for t in range(f):
+            length = len_start + t + 1
+            for li, ly in enumerate(layers):
+                for hx, dx in zip(h_dec[t], d_dec[t]):
+                    dx.copy_(hx, non_blocking=True)
+                q, kn, vn = d_dec[t]
+                resa.decode_sparse(q, kn, vn, ly["k"], ly["v"], ly["desc"], length, spec.r,
+                                   spec.n_min, 1.0, out, ws[li])
+                h_out[li, t].copy_(out, non_blocking=True)
+        for li, ly in enumerate(layers):
+            for hx, dx in zip(h_rect, d_rect):
+                dx.copy_(hx, non_blocking=True)
+            resa.rectify(d_rect[0], d_rect[1], d_rect[2], ly["k"], ly["v"], ly["desc"],
+                         len_start + f, f, 1.0, out_f, ws[li])
+            h_out_f[li].copy_(out_f, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        n = max(2, min(args.steps, 10))
+        t0.record(stream)
+        for _ in range(n):
+            step()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    return {"ms_per_step": t0.elapsed_time(t1) / n, "h2d": h2d, "d2h": d2h}
+
+
+# ----------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload. One sample step is
+    one decode step of the whole batch plus the rectification of one (batch,
+    KV head) group, the latter scaled by the number of groups; amortised over
+    f it gives microseconds per decode step in the benchmark's unit."""
+
+    def __init__(self, spec):
+        import oracle as orc
+        from workload import make_cache
+        self.orc = orc
+        self.spec = spec
+        try:
+            from threadpoolctl import threadpool_info
+            self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            self.threads = os.cpu_count() or 1
+        K, V = make_cache(spec)
+        self.st = orc.State(K, V, spec.len0, spec.group)
+        self.groups = spec.batch * spec.n_kv_heads
+        self.n = 0
+
+    def step(self):
+        from workload import decode_inputs, rectify_inputs
+        spec, st, orc = self.spec, self.st, self.orc
+        q, kn, vn = decode_inputs(spec, self.n % spec.steps)
+        t0 = time.perf_counter()
+        st.decode(q, kn, vn, spec.r, spec.n_min, 1.0)
+        dec_s = time.perf_counter() - t0
+        f, G = spec.f, spec.group
+        q_f, k_f, v_f = rectify_inputs(spec, 0, st.length, f)
+        sub = orc.State.__new__(orc.State)
+        sub.K, sub.V = st.K[:1, :1].copy(), st.V[:1, :1].copy()
+        sub.lo, sub.hi = st.lo[:1, :1].copy(), st.hi[:1, :1].copy()
+        sub.length, sub.group = st.length, G
+        t0 = time.perf_counter()
+        sub.rectify(q_f[:1, :, :G], k_f[:1, :, :1], v_f[:1, :, :1], f, 1.0)
+        rect_s = (time.perf_counter() - t0) * self.groups
+        self.n += 1
+        return (dec_s + rect_s / f) * 1e6
+
+    def describe(self, steps):
+        return (f"{steps} sample steps, each = 1 oracle decode step (whole batch) + rectify of 1 "
+                f"of {self.groups} (batch, KV head) groups scaled x{self.groups}, amortised over "
+                f"f={self.spec.f}; context {self.spec.len0}")
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle as it stands, timed on this host's cores."""
+    from workload import config
+    cfg_idx = WORKLOADS[args.workload]
+    over = {"steps": 64}
+    if args.r is not None:
+        over["r"] = args.r
+    spec = config(cfg_idx, **over)
+    if rank != 0:
+        return None
+    smp = OracleSample(spec)
+    for _ in range(args.warmup):
+        smp.step()
+    per = [smp.step() for _ in range(args.steps)]
+    us = statistics.median(per)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(us * spec.f * args.layers / 1000.0, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) + block means; no dataset, no weights)",
+        "config": {"workload": WORKLOAD_NAMES[cfg_idx], "batch": spec.batch,
+                   "context": spec.len0, "r": spec.r, "f": spec.f, "layers": args.layers},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us", "cores": smp.threads,
+                         "kind": "oracle", "sample": smp.describe(args.steps)},
+        "e2e": {"value": round(us, 1), "unit": "us", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res, spec = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSample(spec)
+        smp.step()                       # warm-up (page-in, BLAS threads)
+        per = [smp.step() for _ in range(3)]
+        res["cpu_baseline"] = {"value": round(statistics.median(per), 1), "unit": "us",
+                               "cores": smp.threads, "kind": "oracle",
+                               "sample": smp.describe(3)}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

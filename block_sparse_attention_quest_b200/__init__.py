@@ -5,7 +5,7 @@ device pointers, sizes and the current CUDA stream to the C ABI declared in
 include/resa.h, and raises on a non-zero status. All arithmetic happens in the
 library's CUDA kernels. PyTorch provides device memory and streams.
 
-The library must be built (``python -m block_sparse_attention_quest_b200.build``
+The library must be built (``python block_sparse_attention_quest_b200/build.py``
 or ``__graft_entry__.build()``); importing this module fails loudly when
 libresa.so is missing. There is no fallback implementation.
 """
@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libresa.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libresa.so not found at {LIB_PATH}; build it with "
-        "`python -m block_sparse_attention_quest_b200.build`")
+        "`python block_sparse_attention_quest_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 RESA_OK = 0
@@ -32,12 +32,14 @@ RESA_ERR_CAPACITY = -3
 RESA_ERR_WORKSPACE = -4
 RESA_ERR_CUDA = -5
 RESA_ERR_TIMEOUT = -6
+RESA_ERR_BAD_INDEX = -7
 RESA_F32 = 0
 RESA_BF16 = 1
 BLOCK = 16
 
 EXPORTED = ("resa_num_selected", "resa_workspace_bytes", "resa_build_desc",
-            "resa_decode_sparse", "resa_decode_dense", "resa_rectify",
+            "resa_decode_sparse", "resa_select_blocks", "resa_attend_blocks",
+            "resa_decode_dense", "resa_rectify",
             "resa_workspace_status", "resa_status_string")
 
 
@@ -59,6 +61,12 @@ _lib.resa_decode_sparse.restype = ctypes.c_int
 _lib.resa_decode_sparse.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, ctypes.c_int64,
                                     ctypes.c_double, ctypes.c_int32, ctypes.c_float, _P, _P, _P,
                                     _P, ctypes.c_size_t, _P]
+_lib.resa_select_blocks.restype = ctypes.c_int
+_lib.resa_select_blocks.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, ctypes.c_int64,
+                                    ctypes.c_double, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
+_lib.resa_attend_blocks.restype = ctypes.c_int
+_lib.resa_attend_blocks.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, ctypes.c_int64, _P,
+                                    ctypes.c_int32, ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.resa_decode_dense.restype = ctypes.c_int
 _lib.resa_decode_dense.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, ctypes.c_int64,
                                    ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
@@ -146,6 +154,24 @@ def decode_sparse(q, k_new, v_new, k_cache, v_cache, desc, length: int, r: float
         ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
         _ptr(desc), int(length), float(r), int(n_min), float(softmax_scale), _ptr(out), _ptr(lse),
         _ptr(sel), _ptr(workspace), workspace.numel(), _stream(stream)), "resa_decode_sparse")
+
+
+def select_blocks(q, k_new, v_new, k_cache, v_cache, desc, length: int, r: float, n_min: int,
+                  sel, workspace, stream=None) -> None:
+    dims = dims_for(k_cache, q.shape[1])
+    _check(_lib.resa_select_blocks(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(desc), int(length), float(r), int(n_min), _ptr(sel), _ptr(workspace),
+        workspace.numel(), _stream(stream)), "resa_select_blocks")
+
+
+def attend_blocks(q, k_cache, v_cache, length: int, sel, softmax_scale: float, out, workspace,
+                  lse=None, stream=None) -> None:
+    dims = dims_for(k_cache, q.shape[1])
+    _check(_lib.resa_attend_blocks(
+        ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(length), _ptr(sel),
+        int(sel.shape[-1]), float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream(stream)), "resa_attend_blocks")
 
 
 def decode_dense(q, k_new, v_new, k_cache, v_cache, desc, length: int, softmax_scale: float, out,

@@ -1,6 +1,6 @@
 """Build libresa.so in-tree with nvcc for sm_100a.
 
-Usage: python -m block_sparse_attention_quest_b200.build [--verbose]
+Usage: python block_sparse_attention_quest_b200/build.py [--verbose]
 """
 from __future__ import annotations
 
@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libresa.so")
-SOURCES = ["api.cu", "desc.cu", "select.cu", "attend.cu"]
+SOURCES = ["api.cu", "desc.cu", "select.cu", "attend.cu", "rectify_tc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -16,6 +16,8 @@ constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 // upper bound on co-resident CTAs assumed when sizing split partials
 constexpr int kSplitCtaBound = 1024;
+// largest rectification window (f) a call accepts
+constexpr int kMaxRectifyRows = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -53,20 +55,43 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// 2-D view [B*H*L_max rows][D cols] of a bf16 cache, 16 x 64 boxes, 128-byte swizzle
-bool make_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+// 2-D view [B*H*L_max rows][D cols] of a bf16 cache, (box_rows x 64) boxes,
+// 128-byte swizzle
+bool make_cache_map(CUtensorMap* m, const void* base, const Shape& s, uint32_t box_rows = 16) {
   auto enc = encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(s.D),
                         static_cast<cuuint64_t>(s.B) * s.H * static_cast<cuuint64_t>(s.L_max)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(s.D) * 2};
-  cuuint32_t box[2] = {64, 16};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+// 3-D view [B*f][Hq][D] of bf16 rectify queries; a (64 x G x 128/G) box is
+// one 128-row tile in the order row = query * G + head
+bool make_query_map(CUtensorMap* m, const void* base, const Shape& s, int f) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.Hq),
+                        static_cast<cuuint64_t>(s.B) * static_cast<cuuint64_t>(f)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(s.D) * 2,
+                           static_cast<cuuint64_t>(s.Hq) * s.D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(s.G), static_cast<cuuint32_t>(128 / s.G)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool rectify_on_tensor_cores(const Shape& s) {
+  return s.bf16 && (s.G == 1 || s.G == 2 || s.G == 4 || s.G == 8);
+}
+int rect_mtiles(const Shape& s, int f) { return (f * s.G + 127) / 128; }
 
 int check_dims(const resa_dims* d, Shape* s) {
   if (d == nullptr) return RESA_ERR_INVALID_ARG;
@@ -115,13 +140,18 @@ int64_t split_bound(int64_t units) {
 }
 
 struct WsLayout {
-  size_t scores, sel, part_ml, part_o, total;
+  size_t scores, sel, counters, part_ml, part_o, total;
 };
 
+// Control block and arrival counters come first, at offsets that depend on
+// the dims only: they must stay put (and zero) from call to call. The scratch
+// regions after them are rewritten by every call.
 WsLayout ws_layout(const Shape& s, int64_t len, int32_t f) {
   WsLayout w{};
   const int64_t M = blocks_of(len);
   size_t off = kCtrlBytes;
+  w.counters = off;
+  off = align_up(off + static_cast<size_t>(s.B) * s.H * kMaxRectifyRows * sizeof(int));
   w.scores = off;
   off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(float));
   w.sel = off;
@@ -129,7 +159,10 @@ WsLayout ws_layout(const Shape& s, int64_t len, int32_t f) {
   // decode rows: B*Hq with units B*H; rectify rows: B*f*Hq with units B*H*f
   const int64_t dec = static_cast<int64_t>(s.B) * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H);
   const int64_t fr = f > 0 ? f : 1;
-  const int64_t rec = static_cast<int64_t>(s.B) * fr * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H * fr);
+  int64_t sb = split_bound(static_cast<int64_t>(s.B) * s.H * fr);
+  const int64_t sb_tc = split_bound(static_cast<int64_t>(s.B) * s.H * rect_mtiles(s, static_cast<int>(fr)));
+  if (sb_tc > sb) sb = sb_tc;
+  const int64_t rec = static_cast<int64_t>(s.B) * fr * s.Hq * sb;
   const int64_t rows = dec > rec ? dec : rec;
   w.part_ml = off;
   off = align_up(off + static_cast<size_t>(rows) * 2 * sizeof(float));
@@ -151,6 +184,9 @@ int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int3
   a.q = q; a.R = R; a.len0 = len0; a.sel = sel; a.n_sel = n_sel; a.S = S; a.scale = scale;
   a.part_o = reinterpret_cast<float*>(ws + w.part_o);
   a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  a.counters = reinterpret_cast<int*>(ws + w.counters);
+  a.out = out;
+  a.lse = lse;
   a.ctrl = reinterpret_cast<Ctrl*>(ws);
   a.k = k; a.v = v;
   CUtensorMap tk, tv;
@@ -159,9 +195,7 @@ int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int3
     a.tm_k = &tk;
     a.tm_v = &tv;
   }
-  cudaError_t e = launch_attend(s, a, st);
-  if (e != cudaSuccess) return RESA_ERR_CUDA;
-  return cuda_status(launch_merge(s, R, S, a.part_o, a.part_ml, out, lse, st));
+  return cuda_status(launch_attend(s, a, st));
 }
 
 }  // namespace
@@ -179,7 +213,7 @@ int32_t resa_num_selected(int64_t len, int32_t block_size, double r, int32_t n_m
 
 size_t resa_workspace_bytes(const resa_dims* dims, int64_t len, int32_t f) {
   Shape s;
-  if (check_dims(dims, &s) != RESA_OK || len < 1 || f < 0) return 0;
+  if (check_dims(dims, &s) != RESA_OK || len < 1 || f < 0 || f > kMaxRectifyRows) return 0;
   return ws_layout(s, len, f).total;
 }
 
@@ -211,6 +245,48 @@ static int check_decode_common(const resa_dims* dims, Shape* s, const void* q, c
   return RESA_OK;
 }
 
+int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
+                       const void* v_new, void* k_cache, void* v_cache, void* desc,
+                       int64_t len, double r, int32_t n_min, int32_t* sel, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_decode_common(dims, &s, q, k_new, v_new, k_cache, v_cache, len, q, workspace,
+                               workspace_bytes, 0);
+  if (rc != RESA_OK) return rc;
+  if (!desc || !aligned16(desc) || !sel) return RESA_ERR_INVALID_ARG;
+  if (!(r > 0.0 && r <= 1.0) || n_min < 1) return RESA_ERR_INVALID_ARG;
+  const int num_sms = device_sms();
+  if (num_sms <= 0) return RESA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int M = static_cast<int>(blocks_of(len));
+  const int n = resa_num_selected(len, 16, r, n_min);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout w = ws_layout(s, len, 0);
+  float* scores = reinterpret_cast<float*>(ws + w.scores);
+  cudaError_t e = launch_score(s, q, desc, scores, k_new, v_new, k_cache, v_cache, desc, len,
+                               num_sms, st);
+  if (e != cudaSuccess) return RESA_ERR_CUDA;
+  return cuda_status(launch_select(s, scores, sel, M, n, st));
+}
+
+int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache,
+                       const void* v_cache, int64_t len, const int32_t* sel, int32_t n_sel,
+                       float softmax_scale, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_decode_common(dims, &s, q, nullptr, nullptr, k_cache, v_cache, len, out,
+                               workspace, workspace_bytes, 0);
+  if (rc != RESA_OK) return rc;
+  if (!sel || n_sel < 1 || n_sel > blocks_of(len) || !std::isfinite(softmax_scale))
+    return RESA_ERR_INVALID_ARG;
+  const int num_sms = device_sms();
+  if (num_sms <= 0) return RESA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout w = ws_layout(s, len, 0);
+  return run_attention(s, q, 1, len, sel, n_sel, softmax_scale, k_cache, v_cache, out, lse, ws, w,
+                       num_sms, static_cast<cudaStream_t>(stream));
+}
+
 int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
                        const void* v_new, void* k_cache, void* v_cache, void* desc,
                        int64_t len, double r, int32_t n_min, float softmax_scale, void* out,
@@ -222,23 +298,15 @@ int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
   if (rc != RESA_OK) return rc;
   if (!desc || !aligned16(desc)) return RESA_ERR_INVALID_ARG;
   if (!(r > 0.0 && r <= 1.0) || n_min < 1 || !std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
-  const int num_sms = device_sms();
-  if (num_sms <= 0) return RESA_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int M = static_cast<int>(blocks_of(len));
   const int n = resa_num_selected(len, 16, r, n_min);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
-  float* scores = reinterpret_cast<float*>(ws + w.scores);
   int32_t* selp = sel ? sel : reinterpret_cast<int32_t*>(ws + w.sel);
-
-  cudaError_t e = launch_score(s, q, desc, scores, k_new, v_new, k_cache, v_cache, desc, len,
-                               num_sms, st);
-  if (e != cudaSuccess) return RESA_ERR_CUDA;
-  e = launch_select(s, scores, selp, M, n, st);
-  if (e != cudaSuccess) return RESA_ERR_CUDA;
-  return run_attention(s, q, 1, len, selp, n, softmax_scale, k_cache, v_cache, out, lse, ws, w,
-                       num_sms, st);
+  rc = resa_select_blocks(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, selp,
+                          workspace, workspace_bytes, stream);
+  if (rc != RESA_OK) return rc;
+  return resa_attend_blocks(dims, q, k_cache, v_cache, len, selp, n, softmax_scale, out, lse,
+                            workspace, workspace_bytes, stream);
 }
 
 int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
@@ -271,7 +339,7 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != RESA_OK) return rc;
-  if (f < 1) return RESA_ERR_INVALID_ARG;
+  if (f < 1 || f > kMaxRectifyRows) return RESA_ERR_INVALID_ARG;
   rc = check_decode_common(dims, &s, q_f, k_f, v_f, k_cache, v_cache, len, out_f, workspace,
                                workspace_bytes, f);
   if (rc != RESA_OK) return rc;
@@ -284,6 +352,27 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
   const WsLayout w = ws_layout(s, len, f);
   cudaError_t e = launch_rectify_write(s, k_f, v_f, k_cache, v_cache, desc, len, f, st);
   if (e != cudaSuccess) return RESA_ERR_CUDA;
+  if (rectify_on_tensor_cores(s)) {
+    RectArgs r{};
+    r.B = s.B; r.H = s.H; r.Hq = s.Hq; r.G = s.G; r.D = s.D; r.f = f;
+    r.mtiles = rect_mtiles(s, f);
+    const int units = s.B * s.H * r.mtiles;
+    const int64_t n_tiles = (len + 127) / 128;
+    int64_t S = units >= num_sms ? 1 : num_sms / units;
+    if (S > kMaxSplits) S = kMaxSplits;
+    if (S > n_tiles) S = n_tiles;
+    r.S = static_cast<int>(S);
+    r.len = len; r.L_max = s.L_max; r.scale = softmax_scale; r.out = out_f;
+    r.part_o = reinterpret_cast<float*>(ws + w.part_o);
+    r.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+    r.ctrl = reinterpret_cast<Ctrl*>(ws);
+    CUtensorMap tq, tk, tv;
+    if (!make_query_map(&tq, q_f, s, f) || !make_cache_map(&tk, k_cache, s, 128) ||
+        !make_cache_map(&tv, v_cache, s, 128))
+      return RESA_ERR_CUDA;
+    r.tm_q = &tq; r.tm_k = &tk; r.tm_v = &tv;
+    return cuda_status(launch_rectify_tc(r, st));
+  }
   return run_attention(s, q_f, f, len - f + 1, nullptr, 0, softmax_scale, k_cache, v_cache, out_f,
                        nullptr, ws, w, num_sms, st);
 }
@@ -299,7 +388,7 @@ int resa_workspace_status(void* workspace, void* stream) {
     const int zero = 0;
     if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
       return RESA_ERR_CUDA;
-    return RESA_ERR_TIMEOUT;
+    return (err & kErrTimeout) ? RESA_ERR_TIMEOUT : RESA_ERR_BAD_INDEX;
   }
   return RESA_OK;
 }
@@ -313,6 +402,7 @@ const char* resa_status_string(int status) {
     case RESA_ERR_WORKSPACE: return "workspace too small";
     case RESA_ERR_CUDA: return "CUDA error";
     case RESA_ERR_TIMEOUT: return "device-side wait timed out";
+    case RESA_ERR_BAD_INDEX: return "block id out of range in the selection";
     default: return "unknown status";
   }
 }

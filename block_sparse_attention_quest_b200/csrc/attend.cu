@@ -29,14 +29,19 @@ struct AttnK {
   const int32_t* sel;
   float* part_o;
   float* part_ml;
+  int* counters;     // [B*R*H] arrival counters of the split CTAs (zero between calls)
   Ctrl* ctrl;
   const void* k;
   const void* v;
+  void* out;         // [B*R][Hq][D] in the cache dtype
+  float* lse;        // [B*R][Hq] or nullptr
   int64_t len0;
   int64_t L_max;
   int R, Hq, H, G, n_sel, S;
   float scale_log2;
 };
+
+constexpr int kIdCache = 1024;   // block ids of one CTA kept in shared memory
 
 __device__ __forceinline__ void split_range(const AttnK& a, int s, int64_t len_r, int& i0,
                                             int& i1) {
@@ -45,14 +50,19 @@ __device__ __forceinline__ void split_range(const AttnK& a, int s, int64_t len_r
   i1 = static_cast<int>(static_cast<int64_t>(s + 1) * n / a.S);
 }
 
-// Merge the per-warp (m, l, O) of one CTA through shared memory and write the
-// CTA's partial. sm must hold NW * 8 * (D + 2) floats.
-template <int D, int NW>
-__device__ __forceinline__ void cta_merge_write(const AttnK& a, float* sm, int br, int g,
-                                                int s_idx) {
+// Merge the per-warp (m, l, O) of one CTA through shared memory. With one
+// split the CTA writes the normalised output; otherwise it writes its partial
+// and the last CTA of the (row, group) to arrive merges all S partials
+// (log-sum-exp weights) into the output and resets the arrival counter.
+// sm must hold NW * 8 * (D + 2) floats; it is reused by the final merge.
+template <typename T, int D, int NW>
+__device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, int g, int s_idx) {
   float* sm_o = sm;                       // [NW][8][D]
   float* sm_m = sm + NW * 8 * D;          // [NW][8]
   float* sm_l = sm_m + NW * 8;            // [NW][8]
+  __shared__ int s_last;
+  T* out = static_cast<T*>(a.out);
+  const int64_t head0 = static_cast<int64_t>(br) * a.Hq + g * a.G;
   for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
     const int h = idx / D, ch = idx % D;
     float mstar = -INFINITY;
@@ -65,13 +75,91 @@ __device__ __forceinline__ void cta_merge_write(const AttnK& a, float* sm, int b
       o = fmaf(sc, sm_o[(w * 8 + h) * D + ch], o);
       l = fmaf(sc, sm_l[w * 8 + h], l);
     }
-    const int64_t row = (static_cast<int64_t>(br) * a.Hq + g * a.G + h) * a.S + s_idx;
-    a.part_o[row * D + ch] = o;
-    if (ch == 0) {
-      a.part_ml[row * 2] = mstar;
-      a.part_ml[row * 2 + 1] = l;
+    if (a.S == 1) {
+      out[(head0 + h) * D + ch] = Dt<T>::from_f(o / l);
+      if (a.lse != nullptr && ch == 0) a.lse[head0 + h] = (mstar + log2f(l)) * 0.69314718055994531f;
+    } else {
+      const int64_t row = (head0 + h) * a.S + s_idx;
+      a.part_o[row * D + ch] = o;
+      if (ch == 0) {
+        a.part_ml[row * 2] = mstar;
+        a.part_ml[row * 2 + 1] = l;
+      }
     }
   }
+  if (a.S == 1) return;
+  __threadfence();
+  __syncthreads();
+  int* counter = a.counters + static_cast<int64_t>(br) * a.H + g;
+  if (threadIdx.x == 0) s_last = atomicAdd(counter, 1) == a.S - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // last CTA: weights of every split for every head of the group
+  float* w_s = sm;                        // [S][8]
+  float* l_h = sm + kMaxSplits * 8;       // [8]
+  float* m_h = l_h + 8;                   // [8]
+  if (threadIdx.x < a.G) {
+    const int h = threadIdx.x;
+    const float* ml = a.part_ml + (head0 + h) * a.S * 2;
+    float mstar = -INFINITY;
+    for (int sp = 0; sp < a.S; ++sp) mstar = fmaxf(mstar, __ldcg(ml + 2 * sp));
+    float l = 0.f;
+    for (int sp = 0; sp < a.S; ++sp) {
+      const float m = __ldcg(ml + 2 * sp);
+      const float w = m == -INFINITY ? 0.f : exp2f(m - mstar);
+      w_s[sp * 8 + h] = w;
+      l = fmaf(w, __ldcg(ml + 2 * sp + 1), l);
+    }
+    l_h[h] = l;
+    m_h[h] = mstar;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
+    const int h = idx / D, ch = idx % D;
+    const float* po = a.part_o + (head0 + h) * a.S * D + ch;
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+    int sp = 0;
+    for (; sp + 8 <= a.S; sp += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldcg(po + static_cast<int64_t>(sp + u) * D);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u] = fmaf(w_s[(sp + u) * 8 + h], x[u], acc[u]);
+    }
+    for (; sp < a.S; ++sp) acc[0] = fmaf(w_s[sp * 8 + h], __ldcg(po + static_cast<int64_t>(sp) * D), acc[0]);
+    float o = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o += acc[u];
+    out[(head0 + h) * D + ch] = Dt<T>::from_f(o / l_h[h]);
+    if (a.lse != nullptr && ch == 0)
+      a.lse[head0 + h] = (m_h[h] + log2f(l_h[h])) * 0.69314718055994531f;
+  }
+  if (threadIdx.x == 0) *counter = 0;
+}
+
+// Block ids of this CTA's slice of the list, cached in shared memory when the
+// slice fits (always, for the sizes one GPU serves); dense rows need none.
+struct IdCache {
+  const int32_t* sel;   // this (b, g)'s list, or nullptr for dense
+  const int* ids;       // shared copy of sel[i0 .. i1) or nullptr
+  int i0;
+  __device__ __forceinline__ int at(int i) const {
+    if (sel == nullptr) return i;
+    return ids ? ids[i - i0] : sel[i];
+  }
+};
+
+__device__ __forceinline__ IdCache load_ids(const int32_t* selp, int i0, int i1, int* smem_ids) {
+  IdCache c{selp, nullptr, i0};
+  if (selp != nullptr && i1 - i0 <= kIdCache) {
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) smem_ids[i - i0] = selp[i];
+    c.ids = smem_ids;
+  }
+  __syncthreads();
+  return c;
 }
 
 // ---------------------------------------------------------------------- bf16
@@ -91,6 +179,7 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   constexpr int KT = D / 16;                 // k-steps of the QK product, m-tiles of PV
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[NW][STAGES];
+  __shared__ int ids_smem[kIdCache];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
 
@@ -104,6 +193,7 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   const int my_count = span > warp ? (span - warp + NW - 1) / NW : 0;
   const int32_t* selp = a.sel ? a.sel + (static_cast<int64_t>(b) * a.H + g) * a.n_sel : nullptr;
   const int64_t row_base = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
+  const IdCache ids = load_ids(selp, i0, i1, ids_smem);
 
   if (lane == 0) {
     prefetch_tmap(&tmK);
@@ -114,13 +204,15 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   }
   __syncwarp();
 
+  const int m_r = static_cast<int>((len_r + kBlock - 1) / kBlock);
+  // block id of this warp's k-th block; ids outside [0, m_r) come back as -1
   auto block_of = [&](int k) -> int {
-    const int i = i0 + warp + k * NW;
-    return selp ? selp[i] : i;
+    const int j = ids.at(i0 + warp + k * NW);
+    return (j >= 0 && j < m_r) ? j : -1;
   };
   auto issue = [&](int k) {
     const int st = k % STAGES;
-    const int j = block_of(k);
+    const int j = max(block_of(k), 0);   // a bad id still completes the stage (block 0)
     const int y = static_cast<int>(row_base + static_cast<int64_t>(j) * kBlock);
     uint8_t* t = tiles + (warp * STAGES + st) * Cfg::kTile;
     mbar_arrive_expect_tx(&bars[warp][st], Cfg::kTile);
@@ -170,8 +262,29 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
     const bool arrived = mbar_wait_bounded(&bars[warp][st], (k / STAGES) & 1, a.ctrl);
     if (!__all_sync(0xffffffffu, arrived)) { ok = false; break; }
     const int j = block_of(k);
+    if (j < 0) {                               // skip the block, report it
+      if (lane == 0) raise_error(a.ctrl, kErrBadIndex);
+      __syncwarp();
+      if (lane == 0 && k + STAGES < my_count) {
+        fence_proxy_async_smem();
+        issue(k + STAGES);
+      }
+      continue;
+    }
     const uint32_t tbase = smem_u32(tiles + (warp * STAGES + st) * Cfg::kTile);
     const uint32_t vbase = tbase + Cfg::kHalves * Cfg::kHalf;
+    const int valid_rows = static_cast<int>(len_r - static_cast<int64_t>(j) * kBlock);
+    if (valid_rows < kBlock) {
+      // slots past the end of the cache: zero their V rows so that 0 * stale
+      // data cannot reach the output
+      uint8_t* vt = tiles + (warp * STAGES + st) * Cfg::kTile + Cfg::kHalves * Cfg::kHalf;
+      for (int idx = lane; idx < Cfg::kHalves * kBlock * 8; idx += 32) {
+        const int hf = idx / (kBlock * 8), rrow = (idx / 8) % kBlock, c = idx % 8;
+        if (rrow >= valid_rows)
+          *reinterpret_cast<uint4*>(vt + hf * Cfg::kHalf + rrow * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
 
     float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -256,7 +369,7 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
     sm_o[(warp * 8 + h1) * D + ch + 8] = o[mt][3];
   }
   __syncthreads();
-  cta_merge_write<D, NW>(a, sm, br, g, s_idx);
+  cta_finish<__nv_bfloat16, D, NW>(a, sm, br, g, s_idx);
 }
 
 // ---------------------------------------------------------------------- fp32
@@ -278,6 +391,8 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
   split_range(a, s_idx, len_r, i0, i1);
   const int32_t* selp = a.sel ? a.sel + (static_cast<int64_t>(b) * a.H + g) * a.n_sel : nullptr;
   const int64_t row_base = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
+  __shared__ int ids_smem[kIdCache];
+  const IdCache ids = load_ids(selp, i0, i1, ids_smem);
   const float* kc = static_cast<const float*>(a.k);
   const float* vc = static_cast<const float*>(a.v);
   float* Ks = tiles + warp * 2 * 16 * P;
@@ -292,15 +407,25 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
     for (int i = 0; i < CPL; ++i) acc[h][i] = 0.f;
   }
   const int t = lane & 15, half = lane >> 4;
+  const int m_r = static_cast<int>((len_r + kBlock - 1) / kBlock);
   for (int i = i0 + warp; i < i1; i += NW) {
-    const int j = selp ? selp[i] : i;
+    const int j = ids.at(i);
+    if (j < 0 || j >= m_r) {                   // skip the block, report it
+      if (lane == 0) raise_error(a.ctrl, kErrBadIndex);
+      continue;
+    }
     const float* kb = kc + (row_base + static_cast<int64_t>(j) * kBlock) * D;
     const float* vb = vc + (row_base + static_cast<int64_t>(j) * kBlock) * D;
     __syncwarp();
+    const int valid_rows = static_cast<int>(len_r - static_cast<int64_t>(j) * kBlock);
     for (int e = lane; e < 16 * D / 4; e += 32) {
       const int row = e / (D / 4), c4 = (e % (D / 4)) * 4;
-      const float4 kv = *reinterpret_cast<const float4*>(kb + row * D + c4);
-      const float4 vv = *reinterpret_cast<const float4*>(vb + row * D + c4);
+      // slots past the end of the cache are never read (their weight is 0)
+      const bool ok_row = row < valid_rows;
+      const float4 kv = ok_row ? *reinterpret_cast<const float4*>(kb + row * D + c4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 vv = ok_row ? *reinterpret_cast<const float4*>(vb + row * D + c4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
       Ks[row * P + c4] = kv.x; Ks[row * P + c4 + 1] = kv.y;
       Ks[row * P + c4 + 2] = kv.z; Ks[row * P + c4 + 3] = kv.w;
       Vs[row * P + c4] = vv.x; Vs[row * P + c4 + 1] = vv.y;
@@ -353,65 +478,12 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
     }
   }
   __syncthreads();
-  cta_merge_write<D, NW>(a, sm, br, g, s_idx);
-}
-
-// ---------------------------------------------------------------------- merge
-template <typename T, int D>
-__global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ part_o,
-                                                    const float* __restrict__ part_ml,
-                                                    T* __restrict__ out, float* __restrict__ lse,
-                                                    int Hq, int S) {
-  constexpr int CPL = D / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int h = blockIdx.x * 4 + warp;
-  if (h >= Hq) return;
-  const int64_t row = static_cast<int64_t>(blockIdx.y) * Hq + h;
-  const float* ml = part_ml + row * S * 2;
-  float ms[2], ls[2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int s = lane + 32 * q;
-    ms[q] = s < S ? ml[2 * s] : -INFINITY;
-    ls[q] = s < S ? ml[2 * s + 1] : 0.f;
-  }
-  float mstar = fmaxf(ms[0], ms[1]);
-  mstar = warp_max_xor(mstar, 16, 1);
-  float w[2], lsum = 0.f;
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    w[q] = ms[q] == -INFINITY ? 0.f : exp2f(ms[q] - mstar);
-    lsum = fmaf(w[q], ls[q], lsum);
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  float acc[CPL];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
-  const float* po = part_o + row * S * D + lane * CPL;
-  for (int s = 0; s < S; ++s) {
-    const float ws = __shfl_sync(0xffffffffu, w[s >> 5], s & 31);
-    if (CPL == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(s) * D);
-      acc[0] = fmaf(ws, x.x, acc[0]);
-      acc[1] = fmaf(ws, x.y, acc[1]);
-      acc[2] = fmaf(ws, x.z, acc[2]);
-      acc[3] = fmaf(ws, x.w, acc[3]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) acc[i] = fmaf(ws, po[static_cast<int64_t>(s) * D + i], acc[i]);
-    }
-  }
-  const float inv = 1.f / lsum;
-  T* orow = out + row * D + lane * CPL;
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) orow[i] = Dt<T>::from_f(acc[i] * inv);
-  if (lse != nullptr && lane == 0) lse[row] = (mstar + log2f(lsum)) * 0.69314718055994531f;
+  cta_finish<float, D, NW>(a, sm, br, g, s_idx);
 }
 
 // ---------------------------------------------------------------------- launch
-constexpr int kNW = 4;
-constexpr int kStages = 3;
+constexpr int kNW = 8;        // warps per CTA (one CTA per SM for bf16)
+constexpr int kStages = 3;    // tiles in flight per warp
 
 template <int D>
 static cudaError_t attend_bf16_t(const Shape& s, const AttnK& k, const AttnArgs& a,
@@ -452,34 +524,17 @@ static cudaError_t attend_f32_t(const Shape& s, const AttnK& k, const AttnArgs& 
   return cudaGetLastError();
 }
 
-int attend_ctas_per_sm(const Shape& s) { return s.bf16 ? 2 : 4; }
+int attend_ctas_per_sm(const Shape& s) { return s.bf16 ? 1 : 2; }
 
 cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st) {
   AttnK k{};
   k.q = a.q; k.sel = a.sel; k.part_o = a.part_o; k.part_ml = a.part_ml; k.ctrl = a.ctrl;
+  k.counters = a.counters; k.out = a.out; k.lse = a.lse;
   k.k = a.k; k.v = a.v; k.len0 = a.len0; k.L_max = s.L_max; k.R = a.R; k.Hq = s.Hq; k.H = s.H;
   k.G = s.G; k.n_sel = a.n_sel; k.S = a.S;
   k.scale_log2 = a.scale * 1.4426950408889634f;
   if (s.bf16) return s.D == 128 ? attend_bf16_t<128>(s, k, a, st) : attend_bf16_t<64>(s, k, a, st);
   return s.D == 128 ? attend_f32_t<128>(s, k, a, st) : attend_f32_t<64>(s, k, a, st);
-}
-
-cudaError_t launch_merge(const Shape& s, int R, int S, const float* part_o, const float* part_ml,
-                         void* out, float* lse, cudaStream_t st) {
-  dim3 grid((s.Hq + 3) / 4, s.B * R);
-  if (s.bf16) {
-    using T = __nv_bfloat16;
-    if (s.D == 128)
-      merge_kernel<T, 128><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<T*>(out), lse, s.Hq, S);
-    else
-      merge_kernel<T, 64><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<T*>(out), lse, s.Hq, S);
-  } else {
-    if (s.D == 128)
-      merge_kernel<float, 128><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<float*>(out), lse, s.Hq, S);
-    else
-      merge_kernel<float, 64><<<grid, 128, 0, st>>>(part_o, part_ml, static_cast<float*>(out), lse, s.Hq, S);
-  }
-  return cudaGetLastError();
 }
 
 }  // namespace resa

@@ -12,7 +12,8 @@ namespace resa {
 
 constexpr int kBlock = 16;             // tokens per block (b)
 constexpr int kCtrlBytes = 256;        // workspace control block
-constexpr int kErrTimeout = 1;         // bit in the control block's error word
+constexpr int kErrTimeout = 1;         // bits of the control block's error word
+constexpr int kErrBadIndex = 2;
 // A device wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 

@@ -45,6 +45,9 @@ struct AttnArgs {
   float scale;            // softmax scale (natural units)
   float* part_o;          // [B*R*Hq][S][D]
   float* part_ml;         // [B*R*Hq][S][2]  (max in log2 units, sum)
+  int* counters;          // [B*R*H], zero between calls
+  void* out;              // [B*R][Hq][D] in the cache dtype
+  float* lse;             // [B*R][Hq] or nullptr
   Ctrl* ctrl;
   const CUtensorMap* tm_k;  // bf16 only (host copies, passed by value to the kernel)
   const CUtensorMap* tm_v;
@@ -52,11 +55,22 @@ struct AttnArgs {
   const void* v;
 };
 cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st);
-int attend_ctas_per_sm(const Shape& s);
 
-// out: [B*R][Hq][D] in the cache dtype; lse: [B*R][Hq] or nullptr
-cudaError_t launch_merge(const Shape& s, int R, int S, const float* part_o, const float* part_ml,
-                         void* out, float* lse, cudaStream_t st);
+// rectification attention on tcgen05 (bf16, group size 1, 2, 4 or 8)
+struct RectArgs {
+  int B, H, Hq, G, D, f, S, mtiles;
+  int64_t len, L_max;
+  float scale;
+  void* out;              // [B][f][Hq][D] bf16
+  float* part_o;          // [B*f*Hq][S][D]
+  float* part_ml;         // [B*f*Hq][S][2]
+  Ctrl* ctrl;
+  const CUtensorMap* tm_q;  // q_f as [B*f][Hq][D], 64 x G x (128/G) boxes
+  const CUtensorMap* tm_k;  // cache as [B*H*L_max][D], 64 x 128 boxes
+  const CUtensorMap* tm_v;
+};
+cudaError_t launch_rectify_tc(const RectArgs& r, cudaStream_t st);
+int attend_ctas_per_sm(const Shape& s);
 
 constexpr int kMaxSplits = 64;
 

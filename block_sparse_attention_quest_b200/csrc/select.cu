@@ -95,6 +95,29 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(b) * a.H + g;
+  const int last_scored = a.M - 1;                 // block M-1 is forced, not scored
+  const int j_begin = blockIdx.x * a.blocks_per_cta;
+  const int j_end = min(j_begin + a.blocks_per_cta, last_scored);
+  const T* dbase = static_cast<const T*>(a.desc) + bh * a.Mmax * 2 * D;
+  float* sout = a.scores + bh * a.M;
+  const int seg = lane / W;
+
+  uint4 raw[U][CPL];
+  auto load_batch = [&](int j0) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * BPL + seg;
+#pragma unroll
+      for (int w = 0; w < CPL; ++w)
+        raw[u][w] = j < j_end ? ld_stream16(dbase + static_cast<int64_t>(j) * 2 * D +
+                                            ((lane % W) + w * W) * CH)
+                              : make_uint4(0, 0, 0, 0);
+    }
+  };
+  // the first descriptor loads go out before the coefficient set-up
+  int j0 = j_begin + warp * U * BPL;
+  if (j0 < j_end) load_batch(j0);
+
   const T* q = static_cast<const T*>(a.q) + (static_cast<int64_t>(b) * a.H * a.G + g * a.G) * D;
   if (tid < D) {
     float n = 0.f, p = 0.f;
@@ -115,24 +138,7 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
 #pragma unroll
     for (int e = 0; e < CH; ++e) cf[w][e] = coef[((lane % W) + w * W) * CH + e];
 
-  const int last_scored = a.M - 1;                 // block M-1 is forced, not scored
-  const int j_begin = blockIdx.x * a.blocks_per_cta;
-  const int j_end = min(j_begin + a.blocks_per_cta, last_scored);
-  const T* dbase = static_cast<const T*>(a.desc) + bh * a.Mmax * 2 * D;
-  float* sout = a.scores + bh * a.M;
-  const int seg = lane / W;
-
-  for (int j0 = j_begin + warp * U * BPL; j0 < j_end; j0 += NW * U * BPL) {
-    uint4 raw[U][CPL];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int j = j0 + u * BPL + seg;
-#pragma unroll
-      for (int w = 0; w < CPL; ++w)
-        raw[u][w] = j < j_end ? ld_stream16(dbase + static_cast<int64_t>(j) * 2 * D +
-                                            ((lane % W) + w * W) * CH)
-                              : make_uint4(0, 0, 0, 0);
-    }
+  for (; j0 < j_end; j0 += NW * U * BPL) {
     float v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -146,6 +152,7 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
       }
       v[u] = acc;
     }
+    if (j0 + NW * U * BPL < j_end) load_batch(j0 + NW * U * BPL);
     transpose_reduce<U, W>(v, lane);
     if (seg_value_owner<U, W>(lane)) {
       const int u = seg_value_index<U, W>(lane);
@@ -176,10 +183,21 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
 template <typename T, int D>
 static cudaError_t score_t(const Shape& s, const ScoreArgs& a0, int num_sms, cudaStream_t st) {
   ScoreArgs a = a0;
+  static int occ[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (occ[dev] == 0) {
+    int o = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_kernel<T, D>, 256, 0);
+    if (e != cudaSuccess) return e;
+    occ[dev] = o > 0 ? o : 1;
+  }
   const int scored = a.M - 1;
   const int units = s.B * s.H;
-  // about 4 resident CTAs per SM, each CTA a multiple of one warp pass
-  const int target = max(1, (4 * num_sms + units - 1) / units);
+  // one wave: every CTA resident at once, each a multiple of one warp pass
+  const int slots = occ[dev] * num_sms;
+  const int target = max(1, slots / units);
   int bpc = (scored + target - 1) / target;
   constexpr int BPL = 32 / ((2 * D / Chunk<T>::N) < 32 ? (2 * D / Chunk<T>::N) : 32);
   const int quantum = 8 * BPL;                     // blocks of one warp-wide U-load
@@ -249,63 +267,98 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t x, uint32_t* w
   return r;
 }
 
-// Grid (H, B). Keeps block M-1 (key forced to the maximum) and the n-1 best
-// other blocks; among equal scores the lower index wins. Output ascending.
+// Grid (H, B). Keeps block M-1 and the n-1 best of blocks 0 .. M-2; among
+// equal scores the lower index wins. Output ascending.
+//
+// Radix select over the keys' offsets from their minimum: the digits start at
+// the highest bit in which the keys differ, so the first histogram is spread
+// over its 256 bins even when every score has the same sign and exponent, and
+// plain shared-memory atomics see little contention.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores,
                                                              int32_t* __restrict__ sel, int H,
                                                              int M, int n, int keys_in_smem) {
   extern __shared__ uint32_t skeys[];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t s_prefix, s_remaining, s_total;
-  const int tid = threadIdx.x;
+  __shared__ uint32_t red_min[32], red_max[32];
+  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_done;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
   const float* s = scores + bh * M;
   int32_t* out = sel + bh * n;
+  const int Mo = M - 1;                            // candidates: blocks 0 .. M-2
+  const int need = n - 1;                          // how many of them to keep
 
-  if (n >= M) {                                    // every block is selected
+  if (need >= Mo) {                                // every block is selected
     for (int j = tid; j < M; j += blockDim.x) out[j] = j;
     return;
   }
-  auto key_at = [&](int j) -> uint32_t {
-    if (keys_in_smem) return skeys[j];
-    return j == M - 1 ? 0xffffffffu : score_key(s[j]);
-  };
-  if (keys_in_smem) {
-    for (int j = tid; j < M; j += blockDim.x) skeys[j] = j == M - 1 ? 0xffffffffu : score_key(s[j]);
+  if (need <= 0) {
+    if (tid == 0) out[0] = M - 1;
+    return;
   }
-  if (tid == 0) { s_prefix = 0u; s_remaining = static_cast<uint32_t>(n); }
+  auto key_at = [&](int j) -> uint32_t { return keys_in_smem ? skeys[j] : score_key(s[j]); };
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int j0 = tid; j0 < Mo; j0 += 8 * kSelThreads) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * kSelThreads;
+      x[u] = j < Mo ? __ldcg(s + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * kSelThreads;
+      if (j < Mo) {
+        const uint32_t k = score_key(x[u]);
+        if (keys_in_smem) skeys[j] = k;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) { red_min[warp] = kmin; red_max[warp] = kmax; }
   __syncthreads();
-
-  const int iters = (M + blockDim.x - 1) / blockDim.x;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    uint32_t a = lane < nw ? red_min[lane] : 0xffffffffu;
+    uint32_t b = lane < nw ? red_max[lane] : 0u;
+    a = __reduce_min_sync(0xffffffffu, a);
+    b = __reduce_max_sync(0xffffffffu, b);
+    if (lane == 0) {
+      s_kmin = a; s_kmax = b;
+      s_prefix = 0u; s_remaining = static_cast<uint32_t>(need); s_done = 0u;
+    }
+  }
+  __syncthreads();
+  const uint32_t base = s_kmin;
+  const uint32_t range = s_kmax - base;
+  // radix passes over rel = key - base, from the top differing bit down
+  int top = 32 - __clz(range);                     // bits of rel that can differ
+  while (top > 0) {
+    const int shift = top > 8 ? top - 8 : 0;
+    const int width = top - shift;
     if (tid < 256) hist[tid] = 0u;
     __syncthreads();
-    const uint32_t prefix = s_prefix;
-    for (int it = 0; it < iters; ++it) {
-      const int j = it * blockDim.x + tid;
-      uint32_t digit = 256u;                       // 256 = not counted
-      if (j < M) {
-        const uint32_t kk = key_at(j);
-        if ((kk & hi_mask) == prefix) digit = (kk >> shift) & 255u;
-      }
-      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      const int leader = __ffs(peers) - 1;
-      if ((tid & 31) == leader && digit < 256u) atomicAdd(&hist[digit], __popc(peers));
+    const uint32_t prefix = s_prefix;              // fixed bits above `top`
+    const uint32_t hi_mask = top >= 32 ? 0u : ~((1u << top) - 1u);
+    for (int j = tid; j < Mo; j += blockDim.x) {
+      const uint32_t rel = key_at(j) - base;
+      if ((rel & hi_mask) == prefix) atomicAdd(&hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
     }
     __syncthreads();
-    if (tid < 32) {
+    if (warp == 0) {
       // lane l owns bins 255-8l .. 248-8l, scanned from the top
       uint32_t c[8], local = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * tid - i]; local += c[i]; }
+      for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * lane - i]; local += c[i]; }
       uint32_t inc = local;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (tid >= o) inc += y;
+        if (lane >= o) inc += y;
       }
       const uint32_t before = inc - local;
       const uint32_t rem = s_remaining;
@@ -314,39 +367,52 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (acc < rem && rem <= acc + c[i]) {
-            s_prefix = prefix | (static_cast<uint32_t>(255 - 8 * tid - i) << shift);
+            const uint32_t digit = static_cast<uint32_t>(255 - 8 * lane - i);
+            s_prefix = prefix | (digit << shift);
             s_remaining = rem - acc;
+            // the whole bin is needed: every key at or above its floor is kept
+            if (rem - acc == c[i]) s_done = 1u;
           }
           acc += c[i];
         }
       }
     }
     __syncthreads();
+    top = s_done ? 0 : shift;
   }
-  const uint32_t T = s_prefix;
-  const uint32_t need_eq = s_remaining;            // keys equal to T to take, lowest index first
+  const uint32_t T = s_prefix;                     // rel threshold
+  const bool whole_bin = s_done != 0u;
+  const uint32_t need_eq = s_remaining;            // rel == T keys to take, lowest index first
 
-  // each thread owns a contiguous run of indices
-  const int per = (M + blockDim.x - 1) / blockDim.x;
-  const int j0 = min(M, tid * per), j1 = min(M, j0 + per);
-  uint32_t n_eq = 0;
-  for (int j = j0; j < j1; ++j) n_eq += key_at(j) == T;
-  const uint32_t eq_before = block_exclusive_scan(n_eq, warp_tot, &s_total);
-  uint32_t n_sel = 0, seen = eq_before;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t kk = key_at(j);
-    if (kk > T) ++n_sel;
-    else if (kk == T) { if (seen < need_eq) ++n_sel; ++seen; }
+  const int per = (Mo + blockDim.x - 1) / blockDim.x;
+  const int j0 = min(Mo, tid * per), j1 = min(Mo, j0 + per);
+  uint32_t n_sel = 0, seen = 0, n_eq = 0;
+  if (whole_bin) {
+    for (int j = j0; j < j1; ++j) n_sel += (key_at(j) - base) >= T;
+  } else {
+    for (int j = j0; j < j1; ++j) n_eq += (key_at(j) - base) == T;
+    seen = block_exclusive_scan(n_eq, warp_tot, &s_total);
+    const uint32_t eq_before = seen;
+    for (int j = j0; j < j1; ++j) {
+      const uint32_t rel = key_at(j) - base;
+      if (rel > T) ++n_sel;
+      else if (rel == T) { if (seen < need_eq) ++n_sel; ++seen; }
+    }
+    seen = eq_before;
   }
   uint32_t pos = block_exclusive_scan(n_sel, warp_tot, &s_total);
-  seen = eq_before;
   for (int j = j0; j < j1; ++j) {
-    const uint32_t kk = key_at(j);
-    bool take = false;
-    if (kk > T) take = true;
-    else if (kk == T) { take = seen < need_eq; ++seen; }
+    const uint32_t rel = key_at(j) - base;
+    bool take;
+    if (whole_bin) {
+      take = rel >= T;
+    } else {
+      take = rel > T;
+      if (rel == T) { take = seen < need_eq; ++seen; }
+    }
     if (take) out[pos++] = j;
   }
+  if (tid == 0) out[need] = M - 1;
 }
 
 cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int M, int n,

@@ -38,9 +38,10 @@
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
  *     only enqueues work on it and returns; nothing synchronises.
  *   - `workspace` is caller-provided device scratch of at least
- *     resa_workspace_bytes() bytes, 256-byte aligned. Its first 256 bytes are
- *     a control block: zero them once before first use. Calls that share one
- *     workspace must be ordered on one stream.
+ *     resa_workspace_bytes() bytes, 256-byte aligned. Zero all of it once
+ *     before first use: it holds an error word and arrival counters that every
+ *     call leaves at zero again. After a call reports an error, zero it again.
+ *     Calls that share one workspace must be ordered on one stream.
  *   - Arguments are validated on the host before anything is launched; an
  *     invalid argument returns a negative resa_status and launches nothing.
  *     A failed launch returns RESA_ERR_CUDA. A device-side wait that gives up
@@ -70,7 +71,8 @@ typedef enum {
   RESA_ERR_CAPACITY = -3,     /* len > max_len */
   RESA_ERR_WORKSPACE = -4,    /* workspace smaller than resa_workspace_bytes() */
   RESA_ERR_CUDA = -5,         /* a CUDA runtime/driver call or launch failed */
-  RESA_ERR_TIMEOUT = -6       /* a device-side wait gave up (flag in the workspace) */
+  RESA_ERR_TIMEOUT = -6,      /* a device-side wait gave up (flag in the workspace) */
+  RESA_ERR_BAD_INDEX = -7     /* a block id in `sel` was out of range (flag in the workspace) */
 } resa_status;
 
 typedef enum { RESA_F32 = 0, RESA_BF16 = 1 } resa_dtype;
@@ -126,6 +128,25 @@ RESA_API int resa_decode_sparse(const resa_dims* dims, const void* q, const void
                        float* lse, int32_t* sel, void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/* Steps 1-3 of resa_decode_sparse alone (append, group scores, top-n): writes
+ * the ascending block list to `sel` ([batch][n_kv_heads][n], required) with
+ * n = resa_num_selected(len, 16, r, n_min). Together with
+ * resa_attend_blocks this is exactly resa_decode_sparse. */
+RESA_API int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
+                                const void* v_new, void* k_cache, void* v_cache, void* desc,
+                                int64_t len, double r, int32_t n_min, int32_t* sel,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Steps 4-5 of resa_decode_sparse alone: every query head attends over the
+ * tokens (< len) of the n_sel blocks its KV group lists in `sel`
+ * ([batch][n_kv_heads][n_sel], distinct block ids below ceil(len/16), in any
+ * order; 1 <= n_sel <= ceil(len/16)). An id outside that range is skipped and
+ * raises the RESA_ERR_BAD_INDEX flag read by resa_workspace_status(). */
+RESA_API int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache,
+                                const void* v_cache, int64_t len, const int32_t* sel,
+                                int32_t n_sel, float softmax_scale, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Dense decode of the same step: step 1 of resa_decode_sparse (desc may be
  * NULL, then descriptors are not updated), then attention over every token
  * < len. This is the r = 1 comparison arm; it skips scoring and selection. */
@@ -144,15 +165,15 @@ RESA_API int resa_decode_dense(const resa_dims* dims, const void* q, const void*
  *     full block contents;
  *  3. out_f[b][i][h] = causal dense attention of q_f[b][i][h], whose position
  *     is len-f+i, over keys 0 .. len-f+i.
- * Requires 1 <= f <= len. */
+ * Requires 1 <= f <= len and f <= 256. */
 RESA_API int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
                  void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
                  float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
                  void* stream);
 
-/* Synchronises `stream`, then reads and clears the device error flag of the
- * workspace control block. Returns RESA_OK, RESA_ERR_TIMEOUT, or
- * RESA_ERR_CUDA. */
+/* Synchronises `stream`, then reads and clears the device error flags of the
+ * workspace control block. Returns RESA_OK, RESA_ERR_TIMEOUT,
+ * RESA_ERR_BAD_INDEX or RESA_ERR_CUDA. */
 RESA_API int resa_workspace_status(void* workspace, void* stream);
 
 /* Human-readable name of a resa_status value (static string). */

@@ -29,6 +29,7 @@ def _declared():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ("resa_build_desc", "resa_decode_sparse", "resa_rectify", "resa_num_selected",
+              "resa_select_blocks", "resa_attend_blocks",
               "resa_workspace_bytes", "resa_decode_dense", "resa_status_string",
               "resa_workspace_status"):
         assert n in names
@@ -128,6 +129,6 @@ def test_rectify_and_build_desc_reject_invalid_arguments(resa):
 
 
 def test_status_strings(resa):
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert resa.status_string(code) != "unknown status"
     assert resa.status_string(-99) == "unknown status"

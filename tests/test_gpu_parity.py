@@ -124,6 +124,30 @@ def test_rectify_shapes(length, f):
         assert p.desc_matches()
 
 
+def test_rectify_fallback_group_of_three():
+    """bf16 with a group size the tensor-core tile does not take (3)."""
+    spec = Spec(batch=2, n_q_heads=6, n_kv_heads=2, head_dim=128, len0=700, steps=8,
+                dtype="bf16", f=32)
+    p = Pair(spec)
+    for step in range(spec.steps):
+        p.decode(step)
+    p.rectify(32)
+    assert p.desc_matches()
+
+
+def test_stale_cache_slots_do_not_leak():
+    """Slots at or past len hold NaN bit patterns; outputs must not see them."""
+    for dtype in ("bf16", "f32"):
+        spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=1000, steps=6,
+                    dtype=dtype, r=0.1, n_min=4, f=16)
+        p = Pair(spec)
+        p.k[:, :, spec.len0:] = float("nan")
+        p.v[:, :, spec.len0:] = float("nan")
+        for step in range(spec.steps):
+            p.decode(step)
+        p.rectify(16)
+
+
 def test_rectify_softmax_scale_argument():
     spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=300, steps=4,
                 dtype="bf16", f=16)
