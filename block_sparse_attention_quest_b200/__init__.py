@@ -40,7 +40,7 @@ BLOCK = 16
 EXPORTED = ("resa_num_selected", "resa_workspace_bytes", "resa_build_desc",
             "resa_decode_sparse", "resa_select_blocks", "resa_attend_blocks",
             "resa_decode_dense", "resa_rectify",
-            "resa_workspace_status", "resa_status_string")
+            "resa_workspace_status", "resa_status_string", "resa_decode_sparse_noalloc")
 
 
 class Dims(ctypes.Structure):
@@ -73,6 +73,10 @@ _lib.resa_decode_dense.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P,
 _lib.resa_rectify.restype = ctypes.c_int
 _lib.resa_rectify.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, ctypes.c_int64,
                               ctypes.c_int32, ctypes.c_float, _P, _P, ctypes.c_size_t, _P]
+_lib.resa_decode_sparse_noalloc.restype = ctypes.c_int
+_lib.resa_decode_sparse_noalloc.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P,
+                                            ctypes.c_int64, ctypes.c_double, ctypes.c_int32,
+                                            ctypes.c_float, _P, _P, _P, _P]
 _lib.resa_workspace_status.restype = ctypes.c_int
 _lib.resa_workspace_status.argtypes = [_P, _P]
 _lib.resa_status_string.restype = ctypes.c_char_p
@@ -190,6 +194,17 @@ def rectify(q_f, k_f, v_f, k_cache, v_cache, desc, length: int, f: int, softmax_
         ctypes.byref(dims), _ptr(q_f), _ptr(k_f), _ptr(v_f), _ptr(k_cache), _ptr(v_cache),
         _ptr(desc), int(length), int(f), float(softmax_scale), _ptr(out_f), _ptr(workspace),
         workspace.numel(), _stream(stream)), "resa_rectify")
+
+
+def decode_sparse_noalloc(q, k_new, v_new, k_cache, v_cache, desc, length: int, r: float,
+                          n_min: int, softmax_scale: float, out, lse=None, sel=None,
+                          stream=None) -> None:
+    """resa_decode_sparse with the library's own fixed scratch (no workspace)."""
+    dims = dims_for(k_cache, q.shape[1])
+    _check(_lib.resa_decode_sparse_noalloc(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(desc), int(length), float(r), int(n_min), float(softmax_scale), _ptr(out), _ptr(lse),
+        _ptr(sel), _stream(stream)), "resa_decode_sparse_noalloc")
 
 
 def workspace_status(workspace, stream=None) -> int:

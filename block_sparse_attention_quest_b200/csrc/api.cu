@@ -200,6 +200,10 @@ int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int3
 
 }  // namespace
 
+namespace resa {
+size_t workspace_zero_prefix(const Shape& s) { return ws_layout(s, 1, 0).scores; }
+}  // namespace resa
+
 extern "C" {
 
 int32_t resa_num_selected(int64_t len, int32_t block_size, double r, int32_t n_min) {

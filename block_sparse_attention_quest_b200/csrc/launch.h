@@ -74,4 +74,8 @@ int attend_ctas_per_sm(const Shape& s);
 
 constexpr int kMaxSplits = 64;
 
+// Bytes at the start of a workspace that must be zero before a call (the
+// error word and the arrival counters); 0 for invalid dims.
+size_t workspace_zero_prefix(const Shape& s);
+
 }  // namespace resa

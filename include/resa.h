@@ -171,6 +171,30 @@ RESA_API int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_
                  float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/* resa_decode_sparse without a caller-provided workspace. The method has no
+ * counterpart for this call; it exists for callers that cannot allocate
+ * device memory themselves (a framework's caching allocator owns the GPU, a
+ * decode loop captured into CUDA graphs must not allocate, a plugin host only
+ * passes input and output pointers).
+ *  - Scratch is a fixed 16 MiB array inside libresa.so's device memory, held
+ *    by every GPU that loads the library until the process exits. Calls whose
+ *    resa_workspace_bytes(dims, len, 0) exceeds 16 MiB return
+ *    RESA_ERR_WORKSPACE and launch nothing.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call outside any
+ *    stream capture.
+ *  - Each call clears the array's error word and counters on `stream`
+ *    (cudaMemsetAsync), then runs resa_decode_sparse on it. It allocates
+ *    nothing. All calls on a device share the one array: calls that may
+ *    overlap on the GPU (different streams, different threads) race and must
+ *    be serialised by the caller.
+ * Arguments and results are those of resa_decode_sparse. */
+RESA_API int resa_decode_sparse_noalloc(const resa_dims* dims, const void* q, const void* k_new,
+                                        const void* v_new, void* k_cache, void* v_cache,
+                                        void* desc, int64_t len, double r, int32_t n_min,
+                                        float softmax_scale, void* out, float* lse,
+                                        int32_t* sel, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * workspace control block. Returns RESA_OK, RESA_ERR_TIMEOUT,
  * RESA_ERR_BAD_INDEX or RESA_ERR_CUDA. */
