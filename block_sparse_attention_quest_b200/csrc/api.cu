@@ -281,7 +281,7 @@ int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache
   int rc = check_decode_common(dims, &s, q, nullptr, nullptr, k_cache, v_cache, len, out,
                                workspace, workspace_bytes, 0);
   if (rc != RESA_OK) return rc;
-  if (!sel || n_sel < 1 || n_sel > blocks_of(len) || !std::isfinite(softmax_scale))
+  if (!sel || n_sel < 1 || n_sel > blocks_of(len) || !(std::isfinite(softmax_scale) && softmax_scale > 0.f))
     return RESA_ERR_INVALID_ARG;
   const int num_sms = device_sms();
   if (num_sms <= 0) return RESA_ERR_CUDA;
@@ -301,7 +301,7 @@ int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
                                workspace_bytes, 0);
   if (rc != RESA_OK) return rc;
   if (!desc || !aligned16(desc)) return RESA_ERR_INVALID_ARG;
-  if (!(r > 0.0 && r <= 1.0) || n_min < 1 || !std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
+  if (!(r > 0.0 && r <= 1.0) || n_min < 1 || !(std::isfinite(softmax_scale) && softmax_scale > 0.f)) return RESA_ERR_INVALID_ARG;
   const int n = resa_num_selected(len, 16, r, n_min);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
@@ -322,7 +322,7 @@ int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
                                workspace_bytes, 0);
   if (rc != RESA_OK) return rc;
   if (desc && !aligned16(desc)) return RESA_ERR_INVALID_ARG;
-  if (!std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
+  if (!(std::isfinite(softmax_scale) && softmax_scale > 0.f)) return RESA_ERR_INVALID_ARG;
   const int num_sms = device_sms();
   if (num_sms <= 0) return RESA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -348,7 +348,7 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
                                workspace_bytes, f);
   if (rc != RESA_OK) return rc;
   if (!k_f || !desc || !aligned16(desc)) return RESA_ERR_INVALID_ARG;
-  if (f > len || !std::isfinite(softmax_scale)) return RESA_ERR_INVALID_ARG;
+  if (f > len || !(std::isfinite(softmax_scale) && softmax_scale > 0.f)) return RESA_ERR_INVALID_ARG;
   const int num_sms = device_sms();
   if (num_sms <= 0) return RESA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

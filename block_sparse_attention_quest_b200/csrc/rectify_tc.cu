@@ -7,14 +7,19 @@
 // of a real dense contraction: S = Q K^T (M = 128 rows, N = 128 keys,
 // K = head_dim) and O += P V (M = 128, N = head_dim, K = 128 keys).
 //
-// One CTA per (KV split, KV head, batch x 128-row tile); 5 warps:
-//   warps 0-3  one query row per thread (= TMEM lane): read S from TMEM,
-//              causal mask, online softmax in float32, write P (bf16) to
-//              shared memory, rescale O in TMEM when the running maximum
-//              moves by more than 2^8, and write the result at the end;
-//   warp 4     one elected thread issues the TMA copies (Q once, K/V tiles of
-//              128 keys in a two-stage ring) and the tcgen05.mma instructions;
-//              completion is signalled with tcgen05.commit on mbarriers.
+// One CTA per (KV split, KV head, batch x 128-row tile); 9 warps:
+//   warps 0-3 and 4-7  two softmax warpgroups; group w takes the key tiles
+//              t = w (mod 2) with its own S and O accumulators in TMEM and
+//              its own shared-memory stage (K, V, P), so one group's softmax
+//              overlaps the other group's MMAs. One query row per thread
+//              (= TMEM lane): row maximum, causal mask on the tail tiles only,
+//              P = 2^(s * scale - m) written bf16 to shared memory, O rescaled
+//              in TMEM only when the running maximum grows by more than 2^8;
+//              the two groups' (m, l, O) are merged at the end;
+//   warp 8     one thread issues the TMA copies (Q once; K and V of each tile
+//              on separate barriers, so K of tile t+2 loads while tile t is
+//              still in its softmax) and the tcgen05.mma instructions, with
+//              completion signalled by tcgen05.commit on mbarriers.
 // The row order inside a tile is m = i * G + h (query i of head h of the
 // group), which is exactly the layout of q_f[b][i][g*G + h][:] viewed as a
 // 3-D tensor, so Q arrives by one box per 64-channel half.
@@ -43,28 +48,40 @@ struct RectCfg {
   static constexpr int kHalves = D / 64;
   static constexpr int kHalfBytes = 128 * 128;            // [128 rows][64 bf16]
   static constexpr int kQBytes = kHalves * kHalfBytes;
-  static constexpr int kKVBytes = 2 * kHalves * kHalfBytes;
+  static constexpr int kKBytes = kHalves * kHalfBytes;    // K (or V) of one 128-key tile
   static constexpr int kPBytes = 2 * kHalfBytes;          // [128 rows][128 keys]
-  static constexpr int kStages = 2;
-  static constexpr int kSmem = kQBytes + kStages * kKVBytes + kPBytes + 1024;
-  static constexpr uint32_t kTmemCols = 256;              // S: cols 0..127, O: 128..
+  // two stages, one per softmax warpgroup: stage w holds K, V and P of the
+  // tiles t = w (mod 2)
+  static constexpr int kStageBytes = 2 * kKBytes + kPBytes;
+  static constexpr int kSmem = kQBytes + 2 * kStageBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;              // S0 S1 O0 O1, 128 columns each
 };
 
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int D>
-__global__ void __launch_bounds__(160, 1) rectify_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                             const __grid_constant__ CUtensorMap tmK,
                                                             const __grid_constant__ CUtensorMap tmV,
                                                             RectK a) {
   using C = RectCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_s, bar_p, bar_pv;
-  __shared__ __align__(8) uint64_t bar_full[C::kStages], bar_empty[C::kStages];
+  __shared__ __align__(8) uint64_t bar_q;
+  __shared__ __align__(8) uint64_t bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
+  __shared__ __align__(8) uint64_t bar_s[2], bar_p[2], bar_pv[2];
   __shared__ uint32_t tmem_base_sh;
+  __shared__ float s_m1[128], s_l1[128];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = base;
-  uint8_t* sKV = sQ + C::kQBytes;
-  uint8_t* sP = sKV + C::kStages * C::kKVBytes;
+  uint8_t* sStage = sQ + C::kQBytes;
+  auto sK = [&](int w) { return sStage + w * C::kStageBytes; };
+  auto sV = [&](int w) { return sStage + w * C::kStageBytes + C::kKBytes; };
+  auto sP = [&](int w) { return sStage + w * C::kStageBytes + 2 * C::kKBytes; };
 
   const int s_idx = blockIdx.x, g = blockIdx.y;
   const int b = blockIdx.z / a.mtiles, mt = blockIdx.z % a.mtiles;
@@ -77,13 +94,15 @@ __global__ void __launch_bounds__(160, 1) rectify_tc_kernel(const __grid_constan
 
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
-    mbar_init(&bar_s, 1);
-    mbar_init(&bar_p, 128);
-    mbar_init(&bar_pv, 1);
 #pragma unroll
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bar_kfull[w], 1);
+      mbar_init(&bar_kempty[w], 1);
+      mbar_init(&bar_vfull[w], 1);
+      mbar_init(&bar_vempty[w], 1);
+      mbar_init(&bar_s[w], 1);
+      mbar_init(&bar_p[w], 128);
+      mbar_init(&bar_pv[w], 1);
     }
     fence_mbar_init();
   }
@@ -92,9 +111,10 @@ __global__ void __launch_bounds__(160, 1) rectify_tc_kernel(const __grid_constan
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  auto tS = [&](int w) { return tmem + 128u * w; };
+  auto tO = [&](int w) { return tmem + 256u + 128u * w; };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ control
     if (lane == 0 && nt > 0) {
       prefetch_tmap(&tmQ);
@@ -107,180 +127,228 @@ __global__ void __launch_bounds__(160, 1) rectify_tc_kernel(const __grid_constan
         tma_load_3d(sQ + hf * C::kHalfBytes, &tmQ, hf * 64, g * a.G, b * a.f + mt * rows_per_q,
                     &bar_q);
       const int64_t row0 = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
-      auto load_kv = [&](int t) {
-        const int st = t % C::kStages;
+      auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int t) {
         const int y = static_cast<int>(row0 + static_cast<int64_t>(t0 + t) * 128);
-        uint8_t* kv = sKV + st * C::kKVBytes;
-        mbar_arrive_expect_tx(&bar_full[st], C::kKVBytes);
+        mbar_arrive_expect_tx(bar, C::kKBytes);
 #pragma unroll
-        for (int hf = 0; hf < C::kHalves; ++hf) {
-          tma_load_2d(kv + hf * C::kHalfBytes, &tmK, hf * 64, y, &bar_full[st]);
-          tma_load_2d(kv + (C::kHalves + hf) * C::kHalfBytes, &tmV, hf * 64, y, &bar_full[st]);
-        }
+        for (int hf = 0; hf < C::kHalves; ++hf) tma_load_2d(dst + hf * C::kHalfBytes, map, hf * 64, y, bar);
       };
-      for (int t = 0; t < nt && t < C::kStages; ++t) load_kv(t);
+      for (int t = 0; t < nt && t < 2; ++t) {
+        load(&tmK, sK(t), &bar_kfull[t], t);
+        load(&tmV, sV(t), &bar_vfull[t], t);
+      }
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false);
       constexpr uint32_t idO = tc::idesc_bf16(128, D, true);
       const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
       auto issue_qk = [&](int t) {
-        const uint32_t k_addr = smem_u32(sKV + (t % C::kStages) * C::kKVBytes);
+        const int w = t & 1;
+        const uint32_t k_addr = smem_u32(sK(w));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc::mma_ss(tS, tc::smem_desc(q_addr + off, 16, 1024), tc::smem_desc(k_addr + off, 16, 1024),
-                     idS, kk > 0);
+          tc::mma_ss(tS(w), tc::smem_desc(q_addr + off, 16, 1024),
+                     tc::smem_desc(k_addr + off, 16, 1024), idS, kk > 0);
         }
-        tc::commit(&bar_s);
+        tc::commit(&bar_s[w]);
+        tc::commit(&bar_kempty[w]);
       };
       auto issue_pv = [&](int t) {
-        const int st = t % C::kStages;
-        const uint32_t v_addr = smem_u32(sKV + st * C::kKVBytes + C::kHalves * C::kHalfBytes);
+        const int w = t & 1;
+        const uint32_t v_addr = smem_u32(sV(w));
+        const uint32_t p_addr = smem_u32(sP(w));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t poff = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc::mma_ss(tO, tc::smem_desc(p_addr + poff, 16, 1024),
-                     tc::smem_desc(v_addr + kk * 2048, C::kHalfBytes, 1024), idO, t > 0 || kk > 0);
+          tc::mma_ss(tO(w), tc::smem_desc(p_addr + poff, 16, 1024),
+                     tc::smem_desc(v_addr + kk * 2048, C::kHalfBytes, 1024), idO, t >= 2 || kk > 0);
         }
-        tc::commit(&bar_pv);
-        tc::commit(&bar_empty[st]);
+        tc::commit(&bar_pv[w]);
+        tc::commit(&bar_vempty[w]);
       };
-      bool ok = mbar_wait_bounded(&bar_q, 0, a.ctrl) && mbar_wait_bounded(&bar_full[0], 0, a.ctrl);
-      if (ok) {
+      bool ok = mbar_wait_bounded(&bar_q, 0, a.ctrl);
+      for (int t = 0; ok && t < nt && t < 2; ++t) {
+        ok = mbar_wait_bounded(&bar_kfull[t], 0, a.ctrl);
+        if (!ok) break;
         tc::fence_after_sync();
-        issue_qk(0);
+        issue_qk(t);
       }
-      for (int t = 1; ok && t <= nt; ++t) {
-        if (!mbar_wait_bounded(&bar_p, (t - 1) & 1, a.ctrl)) { ok = false; break; }
-        tc::fence_after_sync();
-        issue_pv(t - 1);
-        if (t < nt) {
-          if (!mbar_wait_bounded(&bar_full[t % C::kStages], (t / C::kStages) & 1, a.ctrl)) {
-            ok = false;
-            break;
-          }
-          issue_qk(t);
+      for (int t = 0; ok && t < nt; ++t) {
+        const int w = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        const bool refill = t + 2 < nt;
+        // K of tile t is no longer needed once QK(t) completed
+        if (refill) {
+          if (!(ok = mbar_wait_bounded(&bar_kempty[w], ph, a.ctrl))) break;
+          load(&tmK, sK(w), &bar_kfull[w], t + 2);
         }
-        const int refill = t - 1 + C::kStages;
-        if (refill < nt) {
-          const int st = (t - 1) % C::kStages;
-          if (!mbar_wait_bounded(&bar_empty[st], ((t - 1) / C::kStages) & 1, a.ctrl)) {
-            ok = false;
-            break;
-          }
-          load_kv(refill);
+        if (!(ok = mbar_wait_bounded(&bar_p[w], ph, a.ctrl))) break;
+        if (!(ok = mbar_wait_bounded(&bar_vfull[w], ph, a.ctrl))) break;
+        tc::fence_after_sync();
+        issue_pv(t);
+        if (refill) {
+          if (!(ok = mbar_wait_bounded(&bar_vempty[w], ph, a.ctrl))) break;
+          load(&tmV, sV(w), &bar_vfull[w], t + 2);
+          if (!(ok = mbar_wait_bounded(&bar_kfull[w], ph ^ 1, a.ctrl))) break;
+          tc::fence_after_sync();
+          issue_qk(t + 2);
         }
       }
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax rows
-    const int row = threadIdx.x;                          // TMEM lane / tile row
+    // ------------------------------------------------------------ softmax
+    const int w = warp >> 2;                               // warpgroup: tiles t = w (mod 2)
+    const int row = threadIdx.x & 127;                     // TMEM lane / tile row
     const int rg = mt * 128 + row;
     const int qi = rg / a.G, hh = rg % a.G;
     const int64_t qpos = len - a.f + qi;                   // causal limit of this row
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    float m_ref = -INFINITY, l = 0.f;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float sl2 = a.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;                      // reference max (log2 units), sum
     bool ok = true;
-    for (int t = 0; t < nt; ++t) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_s, t & 1, a.ctrl));
+    int u = 0;
+    for (int t = w; t < nt; t += 2, ++u) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_s[w], u & 1, a.ctrl));
       if (!ok) break;
       tc::fence_after_sync();
-      float sv[128];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float chunk[32];
-        tc::ld32(tS + lane_off + c4 * 32, chunk);
-        tc::wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c4 * 32 + i] = chunk[i];
-      }
       const int64_t key0 = static_cast<int64_t>(t0 + t) * 128;
+      // keys above the smallest causal limit of the tile (or past the end of
+      // the cache) exist only in the last tiles
+      const bool masked = key0 + 127 > len - a.f;
+      const int lim = masked ? static_cast<int>(qpos - key0 < 127 ? qpos - key0 : 127) : 127;
+      // pass 1: row maximum of the raw scores
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float z = key0 + c > qpos ? -INFINITY : sv[c] * a.scale_log2;
-        sv[c] = z;
-        mx = fmaxf(mx, z);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tc::ld32(tS(w) + lane_off + c4 * 32, v);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (!masked || c4 * 32 + i <= lim) mx = fmaxf(mx, v[i]);
       }
-      if (t > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_pv, (t - 1) & 1, a.ctrl));
+      mx *= sl2;
+      if (u > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_pv[w], (u - 1) & 1, a.ctrl));
         if (!ok) break;
         tc::fence_after_sync();
       }
-      // new reference maximum only when the row maximum grew by more than 2^8
+      // move the reference only when the row maximum grew by more than 2^8
       const bool need = mx > m_ref + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? mx : m_ref;
-        const float alpha = need ? (m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_new)) : 1.f;
-        if (t > 0) {
+        const float alpha = need ? (m_ref == -INFINITY ? 0.f : ex2(m_ref - m_new)) : 1.f;
+        if (u > 0) {
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             float o[32];
-            tc::ld32(tO + lane_off + c4 * 32, o);
+            tc::ld32(tO(w) + lane_off + c4 * 32, o);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tc::st32(tO + lane_off + c4 * 32, o);
+            tc::st32(tO(w) + lane_off + c4 * 32, o);
           }
           tc::wait_st();
         }
         l *= alpha;
         m_ref = m_new;
       }
-      // P = exp2(s - m_ref) as bf16, K-major with 128-byte swizzle
-      float sum = 0.f;
+      // pass 2: P = 2^(s * scale - m_ref) as bf16 (K-major, 128-byte swizzle)
       const bool live = m_ref != -INFINITY;
+      float sum = 0.f;
+      uint8_t* pw = sP(w);
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        uint32_t w[4];
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tc::ld32(tS(w) + lane_off + c4 * 32, v);
+        tc::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float z0 = sv[c8 * 8 + 2 * e], z1 = sv[c8 * 8 + 2 * e + 1];
-          const float p0 = live && z0 != -INFINITY ? exp2f(z0 - m_ref) : 0.f;
-          const float p1 = live && z1 != -INFINITY ? exp2f(z1 - m_ref) : 0.f;
-          sum += p0 + p1;
-          w[e] = pack_bf16x2(p0, p1);
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t wd[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = c4 * 32 + c8 * 8 + 2 * e;
+            float p0 = ex2(fmaf(v[c8 * 8 + 2 * e], sl2, -m_ref));
+            float p1 = ex2(fmaf(v[c8 * 8 + 2 * e + 1], sl2, -m_ref));
+            if (masked) {
+              if (c > lim) p0 = 0.f;
+              if (c + 1 > lim) p1 = 0.f;
+            }
+            if (!live) { p0 = 0.f; p1 = 0.f; }
+            sum += p0 + p1;
+            wd[e] = pack_bf16x2(p0, p1);
+          }
+          const int chunk = c4 * 4 + c8;                   // 16-byte chunk of 8 keys
+          uint8_t* dst = pw + (chunk >> 3) * C::kHalfBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
-        uint8_t* dst = sP + (c8 >> 3) * C::kHalfBytes + row * 128 + (((c8 & 7) ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       l += sum;
       // V rows past the end of the cache are zeroed (0 * stale data must not
       // reach an output)
       if (key0 + row >= len) {
-        uint8_t* v = sKV + ((t % C::kStages) * C::kKVBytes) + C::kHalves * C::kHalfBytes;
+        uint8_t* v = sV(w);
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf)
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(v + hf * C::kHalfBytes + row * 128 + c * 16) =
-                make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(v + hf * C::kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
-      mbar_arrive(&bar_p);
+      mbar_arrive(&bar_p[w]);
     }
-    if (ok && nt > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_pv, (nt - 1) & 1, a.ctrl));
+    const bool has = u > 0;
+    if (ok && has) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_pv[w], (u - 1) & 1, a.ctrl));
       tc::fence_after_sync();
     }
-    if (ok) {
-      const bool valid = qi < a.f;
-      const int64_t orow = (static_cast<int64_t>(b) * a.f + qi) * a.Hq + g * a.G + hh;
+    // combine the two warpgroups: group 1 hands (m, l, O) over through its own
+    // stage's K/V memory, idle once its last PV product has completed (no
+    // copy targets that stage after group 1's last tile)
+    float* sO1 = reinterpret_cast<float*>(sK(1));            // [128][D], 64 KB at most
+    if (w == 1) {
+      s_m1[row] = has ? m_ref : -INFINITY;
+      s_l1[row] = has ? l : 0.f;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         float o[32];
-        if (nt > 0) {
-          tc::ld32(tO + lane_off + c4 * 32, o);
+        if (has && ok) {
+          tc::ld32(tO(1) + lane_off + c4 * 32, o);
           tc::wait_ld();
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sO1[row * D + ((c4 * 32 + i + row) % D)] = o[i];
+      }
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (w == 0 && ok) {
+      const float m1 = s_m1[row], l1 = s_l1[row];
+      const float m0 = has ? m_ref : -INFINITY, l0 = has ? l : 0.f;
+      const float m = fmaxf(m0, m1);
+      const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
+      const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
+      const float lt = a0 * l0 + a1 * l1;
+      const bool valid = qi < a.f;
+      const int64_t orow = (static_cast<int64_t>(b) * a.f + qi) * a.Hq + g * a.G + hh;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        float o[32];
+        if (has) {
+          tc::ld32(tO(0) + lane_off + c4 * 32, o);
+          tc::wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = a0 * o[i] + a1 * sO1[row * D + ((c4 * 32 + i + row) % D)];
         if (valid) {
           if (a.S == 1) {
-            const float inv = 1.f / l;
+            const float inv = 1.f / lt;
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + orow * D + c4 * 32;
 #pragma unroll
             for (int i = 0; i < 32; i += 2)
@@ -294,8 +362,8 @@ __global__ void __launch_bounds__(160, 1) rectify_tc_kernel(const __grid_constan
         }
       }
       if (valid && a.S > 1) {
-        a.part_ml[(orow * a.S + s_idx) * 2] = m_ref;
-        a.part_ml[(orow * a.S + s_idx) * 2 + 1] = l;
+        a.part_ml[(orow * a.S + s_idx) * 2] = m;
+        a.part_ml[(orow * a.S + s_idx) * 2 + 1] = lt;
       }
     }
   }
@@ -377,7 +445,7 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   k.len = r.len; k.L_max = r.L_max; k.H = r.H; k.Hq = r.Hq; k.G = r.G; k.f = r.f; k.S = r.S;
   k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
   dim3 grid(r.S, r.H, r.B * r.mtiles);
-  rectify_tc_kernel<D><<<grid, 160, C::kSmem, st>>>(*r.tm_q, *r.tm_k, *r.tm_v, k);
+  rectify_tc_kernel<D><<<grid, 288, C::kSmem, st>>>(*r.tm_q, *r.tm_k, *r.tm_v, k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || r.S == 1) return e;
   const int64_t rows = static_cast<int64_t>(r.B) * r.f * r.Hq;

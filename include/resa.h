@@ -34,7 +34,7 @@
  *   - `len` is the number of valid tokens in the cache, counting the token a
  *     decode call appends. All batch rows share one len.
  *   - q, k, v, desc and out share the dtype in resa_dims.dtype; softmax and
- *     accumulation are float32.
+ *     accumulation are float32; softmax_scale must be finite and positive.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
  *     only enqueues work on it and returns; nothing synchronises.
  *   - `workspace` is caller-provided device scratch of at least

@@ -101,6 +101,8 @@ def test_decode_rejects_invalid_arguments(resa):
     assert _decode(resa, d, r=1.01) == E.RESA_ERR_INVALID_ARG
     assert _decode(resa, d, n_min=0) == E.RESA_ERR_INVALID_ARG
     assert _decode(resa, d, scale=float("nan")) == E.RESA_ERR_INVALID_ARG
+    assert _decode(resa, d, scale=-1.0) == E.RESA_ERR_INVALID_ARG
+    assert _decode(resa, d, scale=0.0) == E.RESA_ERR_INVALID_ARG
     assert _decode(resa, d, ws_bytes=1024) == E.RESA_ERR_WORKSPACE
     assert _decode(resa, _dims(resa, head_dim=96)) == E.RESA_ERR_UNSUPPORTED
     assert _decode(resa, _dims(resa, block_size=32)) == E.RESA_ERR_UNSUPPORTED
