@@ -177,7 +177,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? RESA_OK : RESA_ERR_CU
 // split-KV attention over `R` query rows + merge
 int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int32_t* sel, int n_sel,
                   float scale, const void* k, const void* v, void* out, float* lse, uint8_t* ws,
-                  const WsLayout& w, int num_sms, cudaStream_t st) {
+                  const WsLayout& w, int num_sms, cudaStream_t st, bool pdl = false) {
   const int64_t min_blocks = sel ? n_sel : blocks_of(len0);
   const int S = splits_for(s.B * s.H * R, min_blocks, num_sms, s);
   AttnArgs a{};
@@ -189,6 +189,7 @@ int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int3
   a.lse = lse;
   a.ctrl = reinterpret_cast<Ctrl*>(ws);
   a.k = k; a.v = v;
+  a.pdl = pdl;
   CUtensorMap tk, tv;
   if (s.bf16) {
     if (!make_cache_map(&tk, k, s) || !make_cache_map(&tv, v, s)) return RESA_ERR_CUDA;
@@ -259,6 +260,7 @@ int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
   if (rc != RESA_OK) return rc;
   if (!desc || !aligned16(desc) || !sel) return RESA_ERR_INVALID_ARG;
   if (!(r > 0.0 && r <= 1.0) || n_min < 1) return RESA_ERR_INVALID_ARG;
+  if (blocks_of(len) > 262144) return RESA_ERR_UNSUPPORTED;
   const int num_sms = device_sms();
   if (num_sms <= 0) return RESA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -273,10 +275,10 @@ int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
   return cuda_status(launch_select(s, scores, sel, M, n, st));
 }
 
-int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache,
-                       const void* v_cache, int64_t len, const int32_t* sel, int32_t n_sel,
-                       float softmax_scale, void* out, float* lse, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+static int attend_blocks_impl(const resa_dims* dims, const void* q, const void* k_cache,
+                              const void* v_cache, int64_t len, const int32_t* sel, int32_t n_sel,
+                              float softmax_scale, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream, bool pdl) {
   Shape s;
   int rc = check_decode_common(dims, &s, q, nullptr, nullptr, k_cache, v_cache, len, out,
                                workspace, workspace_bytes, 0);
@@ -288,7 +290,15 @@ int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
   return run_attention(s, q, 1, len, sel, n_sel, softmax_scale, k_cache, v_cache, out, lse, ws, w,
-                       num_sms, static_cast<cudaStream_t>(stream));
+                       num_sms, static_cast<cudaStream_t>(stream), pdl);
+}
+
+int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache,
+                       const void* v_cache, int64_t len, const int32_t* sel, int32_t n_sel,
+                       float softmax_scale, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return attend_blocks_impl(dims, q, k_cache, v_cache, len, sel, n_sel, softmax_scale, out, lse,
+                            workspace, workspace_bytes, stream, false);
 }
 
 int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
@@ -309,8 +319,10 @@ int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
   rc = resa_select_blocks(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, selp,
                           workspace, workspace_bytes, stream);
   if (rc != RESA_OK) return rc;
-  return resa_attend_blocks(dims, q, k_cache, v_cache, len, selp, n, softmax_scale, out, lse,
-                            workspace, workspace_bytes, stream);
+  // the attention kernel is a programmatic dependent of the select kernel:
+  // its prologue overlaps the selection, it reads the block list after it
+  return attend_blocks_impl(dims, q, k_cache, v_cache, len, selp, n, softmax_scale, out, lse,
+                            workspace, workspace_bytes, stream, true);
 }
 
 int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,

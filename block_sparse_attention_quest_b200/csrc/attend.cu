@@ -95,47 +95,40 @@ __device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, in
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // last CTA: weights of every split for every head of the group
-  float* w_s = sm;                        // [S][8]
-  float* l_h = sm + kMaxSplits * 8;       // [8]
-  float* m_h = l_h + 8;                   // [8]
-  if (threadIdx.x < a.G) {
-    const int h = threadIdx.x;
-    const float* ml = a.part_ml + (head0 + h) * a.S * 2;
-    float mstar = -INFINITY;
-    for (int sp = 0; sp < a.S; ++sp) mstar = fmaxf(mstar, __ldcg(ml + 2 * sp));
-    float l = 0.f;
-    for (int sp = 0; sp < a.S; ++sp) {
-      const float m = __ldcg(ml + 2 * sp);
-      const float w = m == -INFINITY ? 0.f : exp2f(m - mstar);
-      w_s[sp * 8 + h] = w;
-      l = fmaf(w, __ldcg(ml + 2 * sp + 1), l);
-    }
-    l_h[h] = l;
-    m_h[h] = mstar;
-  }
-  __syncthreads();
+  // last CTA: each thread merges its (head, channel) outputs over all splits.
+  // The partial outputs and the (m, l) pairs of a chunk of up to 32 splits
+  // are loaded together (one round trip to L2) and folded in with an online
+  // log-sum-exp, so no step waits on another load.
   for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
     const int h = idx / D, ch = idx % D;
     const float* po = a.part_o + (head0 + h) * a.S * D + ch;
-    float acc[8];
+    const float* ml = a.part_ml + (head0 + h) * a.S * 2;
+    float run_m = -INFINITY, run_l = 0.f, run_o = 0.f;
+    for (int sp0 = 0; sp0 < a.S; sp0 += 32) {
+      float x[32], mv[32], lv[32];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-    int sp = 0;
-    for (; sp + 8 <= a.S; sp += 8) {
-      float x[8];
+      for (int u = 0; u < 32; ++u) {
+        const bool in = sp0 + u < a.S;
+        x[u] = in ? __ldcg(po + static_cast<int64_t>(sp0 + u) * D) : 0.f;
+        mv[u] = in ? __ldcg(ml + 2 * (sp0 + u)) : -INFINITY;
+        lv[u] = in ? __ldcg(ml + 2 * (sp0 + u) + 1) : 0.f;
+      }
+      float cm = run_m;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = __ldcg(po + static_cast<int64_t>(sp + u) * D);
+      for (int u = 0; u < 32; ++u) cm = fmaxf(cm, mv[u]);
+      const float sc = run_m == -INFINITY ? 0.f : exp2f(run_m - cm);
+      run_o *= sc;
+      run_l *= sc;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc[u] = fmaf(w_s[(sp + u) * 8 + h], x[u], acc[u]);
+      for (int u = 0; u < 32; ++u) {
+        const float w = mv[u] == -INFINITY ? 0.f : exp2f(mv[u] - cm);
+        run_o = fmaf(w, x[u], run_o);
+        run_l = fmaf(w, lv[u], run_l);
+      }
+      run_m = cm;
     }
-    for (; sp < a.S; ++sp) acc[0] = fmaf(w_s[sp * 8 + h], __ldcg(po + static_cast<int64_t>(sp) * D), acc[0]);
-    float o = 0.f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) o += acc[u];
-    out[(head0 + h) * D + ch] = Dt<T>::from_f(o / l_h[h]);
-    if (a.lse != nullptr && ch == 0)
-      a.lse[head0 + h] = (m_h[h] + log2f(l_h[h])) * 0.69314718055994531f;
+    out[(head0 + h) * D + ch] = Dt<T>::from_f(run_o / run_l);
+    if (a.lse != nullptr && ch == 0) a.lse[head0 + h] = (run_m + log2f(run_l)) * 0.69314718055994531f;
   }
   if (threadIdx.x == 0) *counter = 0;
 }
@@ -193,8 +186,6 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   const int my_count = span > warp ? (span - warp + NW - 1) / NW : 0;
   const int32_t* selp = a.sel ? a.sel + (static_cast<int64_t>(b) * a.H + g) * a.n_sel : nullptr;
   const int64_t row_base = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
-  const IdCache ids = load_ids(selp, i0, i1, ids_smem);
-
   if (lane == 0) {
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -203,6 +194,30 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
     fence_mbar_init();
   }
   __syncwarp();
+
+  // q^T as the B operand: lane (gq = lane / 4, c = lane % 4) holds head gq,
+  // channels kk*16 + 2c, +1 (b0) and kk*16 + 8 + 2c, +1 (b1)
+  const int gq = lane >> 2, cq = lane & 3;
+  uint32_t qb[KT][2];
+  {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) +
+                                (static_cast<int64_t>(br) * a.Hq + g * a.G + gq) * D;
+#pragma unroll
+    for (int kk = 0; kk < KT; ++kk) {
+      if (gq < a.G) {
+        qb[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * cq);
+        qb[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * cq);
+      } else {
+        qb[kk][0] = 0u;
+        qb[kk][1] = 0u;
+      }
+    }
+  }
+
+  // Everything above may run before the kernel that produced the block list
+  // has finished (programmatic dependent launch); block ids are read after.
+  grid_dependency_wait();
+  const IdCache ids = load_ids(selp, i0, i1, ids_smem);
 
   const int m_r = static_cast<int>((len_r + kBlock - 1) / kBlock);
   // block id of this warp's k-th block; ids outside [0, m_r) come back as -1
@@ -224,25 +239,6 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   };
   if (lane == 0) {
     for (int k = 0; k < my_count && k < STAGES; ++k) issue(k);
-  }
-
-  // q^T as the B operand: lane (gq = lane / 4, c = lane % 4) holds head gq,
-  // channels kk*16 + 2c, +1 (b0) and kk*16 + 8 + 2c, +1 (b1)
-  const int gq = lane >> 2, cq = lane & 3;
-  uint32_t qb[KT][2];
-  {
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) +
-                                (static_cast<int64_t>(br) * a.Hq + g * a.G + gq) * D;
-#pragma unroll
-    for (int kk = 0; kk < KT; ++kk) {
-      if (gq < a.G) {
-        qb[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * cq);
-        qb[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * cq);
-      } else {
-        qb[kk][0] = 0u;
-        qb[kk][1] = 0u;
-      }
-    }
   }
 
   float o[KT][4];
@@ -392,6 +388,7 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
   const int32_t* selp = a.sel ? a.sel + (static_cast<int64_t>(b) * a.H + g) * a.n_sel : nullptr;
   const int64_t row_base = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
   __shared__ int ids_smem[kIdCache];
+  grid_dependency_wait();
   const IdCache ids = load_ids(selp, i0, i1, ids_smem);
   const float* kc = static_cast<const float*>(a.k);
   const float* vc = static_cast<const float*>(a.v);
@@ -498,9 +495,17 @@ static cudaError_t attend_bf16_t(const Shape& s, const AttnK& k, const AttnArgs&
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(a.S, s.H, s.B * a.R);
-  attend_bf16_kernel<D, kNW, kStages><<<grid, kNW * 32, Cfg::kSmem, st>>>(*a.tm_k, *a.tm_v, k);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.S, s.H, s.B * a.R);
+  cfg.blockDim = dim3(kNW * 32);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attend_bf16_kernel<D, kNW, kStages>, *a.tm_k, *a.tm_v, k);
 }
 
 template <int D>
@@ -519,9 +524,17 @@ static cudaError_t attend_f32_t(const Shape& s, const AttnK& k, const AttnArgs& 
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(a.S, s.H, s.B * a.R);
-  attend_f32_kernel<D, kNW><<<grid, kNW * 32, smem, st>>>(k);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.S, s.H, s.B * a.R);
+  cfg.blockDim = dim3(kNW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attend_f32_kernel<D, kNW>, k);
 }
 
 int attend_ctas_per_sm(const Shape& s) { return s.bf16 ? 1 : 2; }

@@ -53,6 +53,7 @@ struct AttnArgs {
   const CUtensorMap* tm_v;
   const void* k;          // cache base pointers (fp32 path)
   const void* v;
+  bool pdl;               // launched as a programmatic dependent of the select kernel
 };
 cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st);
 

@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   constexpr int NW = 8;
 
   __shared__ float coef[2 * D];                    // [N (for lo) | P (for hi)]
+  grid_launch_dependents();
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(b) * a.H + g;
@@ -102,6 +103,15 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   float* sout = a.scores + bh * a.M;
   const int seg = lane / W;
 
+  // the group's query values go out first: the coefficients need them before
+  // any descriptor can be used, and behind the descriptor stream they would
+  // wait for most of it
+  const T* q = static_cast<const T*>(a.q) + (static_cast<int64_t>(b) * a.H * a.G + g * a.G) * D;
+  float qv[8];
+  if (tid < D) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h) qv[h] = h < a.G ? Dt<T>::to_f(q[h * D + tid]) : 0.f;
+  }
   uint4 raw[U][CPL];
   auto load_batch = [&](int j0) {
 #pragma unroll
@@ -114,17 +124,15 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
                               : make_uint4(0, 0, 0, 0);
     }
   };
-  // the first descriptor loads go out before the coefficient set-up
   int j0 = j_begin + warp * U * BPL;
   if (j0 < j_end) load_batch(j0);
 
-  const T* q = static_cast<const T*>(a.q) + (static_cast<int64_t>(b) * a.H * a.G + g * a.G) * D;
   if (tid < D) {
     float n = 0.f, p = 0.f;
-    for (int h = 0; h < a.G; ++h) {
-      const float x = Dt<T>::to_f(q[h * D + tid]);
-      n += fminf(x, 0.f);
-      p += fmaxf(x, 0.f);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      n += fminf(qv[h], 0.f);
+      p += fmaxf(qv[h], 0.f);
     }
     coef[tid] = n;
     coef[D + tid] = p;
@@ -229,6 +237,9 @@ cudaError_t launch_score(const Shape& s, const void* q, const void* desc, float*
 // ---------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
 constexpr int kSelSmemKeys = 40960;   // keys kept in shared memory up to this M
+constexpr int kSelMaxM = 262144;      // largest block count a selection accepts
+constexpr int kBins = 2048;           // first pass: the top 11 bits of the key offset
+constexpr int kCand = 1024;           // threshold-bin candidates resolved by rank
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -236,8 +247,8 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// exclusive prefix sum over the block (kSelThreads threads); returns the
-// thread's exclusive offset, writes the block total to *total
+// exclusive prefix sum over the block; returns the thread's offset and writes
+// the block total to *total
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t x, uint32_t* warp_tot,
                                                          uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -267,27 +278,65 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t x, uint32_t* w
   return r;
 }
 
+// Sum of x over the block's warps (one value per warp, lane 0 holds it);
+// returns the exclusive prefix of this warp and writes the total.
+__device__ __forceinline__ uint32_t warp_exclusive_offset(uint32_t x, uint32_t* warp_tot,
+                                                          uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    const uint32_t t = lane < nw ? warp_tot[lane] : 0u;
+    uint32_t inc = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane < nw) warp_tot[lane] = inc - t;
+    if (lane == 31) *total = inc;
+  }
+  __syncthreads();
+  const uint32_t r = warp_tot[warp];
+  __syncthreads();
+  return r;
+}
+
 // Grid (H, B). Keeps block M-1 and the n-1 best of blocks 0 .. M-2; among
 // equal scores the lower index wins. Output ascending.
 //
-// Radix select over the keys' offsets from their minimum: the digits start at
-// the highest bit in which the keys differ, so the first histogram is spread
-// over its 256 bins even when every score has the same sign and exponent, and
-// plain shared-memory atomics see little contention.
+// Keys are order-preserving 32-bit images of the scores, taken relative to
+// the group minimum. A first histogram over the top 11 bits of that offset
+// (starting at the highest bit in which the keys differ, so the bins spread
+// even when all scores share sign and exponent) locates the threshold bin;
+// its few candidates are then ranked exactly (key descending, index
+// ascending). When the bin is crowded (near-constant scores) 8-bit radix
+// passes continue on the remaining bits instead. The ascending output is
+// written by warps that each own a contiguous index range and order their
+// lanes with ballots, so every shared-memory read is conflict-free.
+template <bool IN_SMEM>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores,
                                                              int32_t* __restrict__ sel, int H,
-                                                             int M, int n, int keys_in_smem) {
-  extern __shared__ uint32_t skeys[];
-  __shared__ uint32_t hist[256];
+                                                             int M, int n) {
+  extern __shared__ uint32_t dyn[];               // [keys (if in smem)][chosen bitmap]
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t cand_rel[kCand];
+  __shared__ int cand_j[kCand];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t red_min[32], red_max[32];
-  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_done;
+  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand;
+  __shared__ int s_mode;                          // 0 exact threshold, 1 bin floor, 2 ranked bin
+  grid_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
   const float* s = scores + bh * M;
   int32_t* out = sel + bh * n;
   const int Mo = M - 1;                            // candidates: blocks 0 .. M-2
   const int need = n - 1;                          // how many of them to keep
+  uint32_t* skeys = dyn;
+  uint32_t* chosen = dyn + (IN_SMEM ? M : 0);
+  const int nwords = (Mo + 31) >> 5;
 
   if (need >= Mo) {                                // every block is selected
     for (int j = tid; j < M; j += blockDim.x) out[j] = j;
@@ -297,7 +346,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     if (tid == 0) out[0] = M - 1;
     return;
   }
-  auto key_at = [&](int j) -> uint32_t { return keys_in_smem ? skeys[j] : score_key(s[j]); };
+  grid_dependency_wait();                          // scores come from the previous kernel
+  auto key_at = [&](int j) -> uint32_t {
+    if constexpr (IN_SMEM) return skeys[j];
+    else return score_key(__ldcg(s + j));
+  };
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int j0 = tid; j0 < Mo; j0 += 8 * kSelThreads) {
     float x[8];
@@ -311,12 +364,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
       const int j = j0 + u * kSelThreads;
       if (j < Mo) {
         const uint32_t k = score_key(x[u]);
-        if (keys_in_smem) skeys[j] = k;
+        if constexpr (IN_SMEM) skeys[j] = k;
         kmin = min(kmin, k);
         kmax = max(kmax, k);
       }
     }
   }
+  for (int w = tid; w < nwords; w += blockDim.x) chosen[w] = 0u;
+  for (int b = tid; b < kBins; b += blockDim.x) hist[b] = 0u;
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if (lane == 0) { red_min[warp] = kmin; red_max[warp] = kmax; }
@@ -329,28 +384,83 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     b = __reduce_max_sync(0xffffffffu, b);
     if (lane == 0) {
       s_kmin = a; s_kmax = b;
-      s_prefix = 0u; s_remaining = static_cast<uint32_t>(need); s_done = 0u;
+      s_prefix = 0u; s_remaining = static_cast<uint32_t>(need); s_ncand = 0u; s_mode = 0;
     }
   }
   __syncthreads();
   const uint32_t base = s_kmin;
   const uint32_t range = s_kmax - base;
-  // radix passes over rel = key - base, from the top differing bit down
   int top = 32 - __clz(range);                     // bits of rel that can differ
+  const int shift = top > 11 ? top - 11 : 0;
+  if (top > 0) {
+    // ---- first pass: 2048 bins
+    for (int j = tid; j < Mo; j += blockDim.x) atomicAdd(&hist[(key_at(j) - base) >> shift], 1u);
+    __syncthreads();
+    {
+      // thread t owns bins 2047-2t and 2046-2t (descending); a block scan of
+      // the per-thread counts from the top finds the threshold bin
+      const uint32_t c0 = hist[kBins - 1 - 2 * tid], c1 = hist[kBins - 2 - 2 * tid];
+      const uint32_t before = block_exclusive_scan(c0 + c1, warp_tot, &s_total);
+      const uint32_t rem = static_cast<uint32_t>(need);
+      uint32_t acc = before;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t c = e == 0 ? c0 : c1;
+        if (acc < rem && rem <= acc + c) {
+          const uint32_t digit = static_cast<uint32_t>(kBins - 1 - 2 * tid - e);
+          s_prefix = digit << shift;
+          s_remaining = rem - acc;
+          s_mode = (rem - acc == c) ? 1 : (c <= static_cast<uint32_t>(kCand) && shift > 0 ? 2 : 0);
+        }
+        acc += c;
+      }
+    }
+    __syncthreads();
+    top = shift;
+    if (s_mode == 2) {
+      // ---- gather the threshold bin and rank its members exactly
+      const uint32_t bin = s_prefix >> shift;
+      for (int j = tid; j < Mo; j += blockDim.x) {
+        const uint32_t rel = key_at(j) - base;
+        if ((rel >> shift) == bin) {
+          const uint32_t slot = atomicAdd(&s_ncand, 1u);
+          cand_rel[slot] = rel;
+          cand_j[slot] = j;
+        }
+      }
+      __syncthreads();
+      const int c = static_cast<int>(s_ncand);
+      const uint32_t take = s_remaining;
+      for (int i = tid; i < c; i += blockDim.x) {
+        const uint32_t r = cand_rel[i];
+        const int jj = cand_j[i];
+        uint32_t rank = 0;
+        for (int k = 0; k < c; ++k) {
+          const uint32_t rk = cand_rel[k];
+          rank += (rk > r) || (rk == r && cand_j[k] < jj);
+        }
+        if (rank < take) atomicOr(&chosen[jj >> 5], 1u << (jj & 31));
+      }
+      __syncthreads();
+      top = 0;
+    } else if (s_mode == 1) {
+      top = 0;
+    }
+  }
+  // ---- remaining 8-bit radix passes (crowded threshold bin)
   while (top > 0) {
-    const int shift = top > 8 ? top - 8 : 0;
-    const int width = top - shift;
+    const int sh = top > 8 ? top - 8 : 0;
+    const int width = top - sh;
     if (tid < 256) hist[tid] = 0u;
     __syncthreads();
-    const uint32_t prefix = s_prefix;              // fixed bits above `top`
+    const uint32_t prefix = s_prefix;
     const uint32_t hi_mask = top >= 32 ? 0u : ~((1u << top) - 1u);
     for (int j = tid; j < Mo; j += blockDim.x) {
       const uint32_t rel = key_at(j) - base;
-      if ((rel & hi_mask) == prefix) atomicAdd(&hist[(rel >> shift) & ((1u << width) - 1u)], 1u);
+      if ((rel & hi_mask) == prefix) atomicAdd(&hist[(rel >> sh) & ((1u << width) - 1u)], 1u);
     }
     __syncthreads();
     if (warp == 0) {
-      // lane l owns bins 255-8l .. 248-8l, scanned from the top
       uint32_t c[8], local = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * lane - i]; local += c[i]; }
@@ -367,70 +477,339 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (acc < rem && rem <= acc + c[i]) {
-            const uint32_t digit = static_cast<uint32_t>(255 - 8 * lane - i);
-            s_prefix = prefix | (digit << shift);
+            s_prefix = prefix | (static_cast<uint32_t>(255 - 8 * lane - i) << sh);
             s_remaining = rem - acc;
-            // the whole bin is needed: every key at or above its floor is kept
-            if (rem - acc == c[i]) s_done = 1u;
+            if (rem - acc == c[i]) s_mode = 1;
           }
           acc += c[i];
         }
       }
     }
     __syncthreads();
-    top = s_done ? 0 : shift;
+    top = s_mode == 1 ? 0 : sh;
   }
-  const uint32_t T = s_prefix;                     // rel threshold
-  const bool whole_bin = s_done != 0u;
-  const uint32_t need_eq = s_remaining;            // rel == T keys to take, lowest index first
+  // ---- ascending compaction, one contiguous index range per warp
+  // mode 0: rel > T, plus the need_eq lowest-index keys with rel == T
+  // mode 1: rel >= T (the floor of a bin that is taken whole)
+  // mode 2: rel at or above the floor of the next bin, plus ranked members
+  const int mode = s_mode;
+  const uint32_t T = s_prefix;
+  const uint64_t next_floor = static_cast<uint64_t>(T) + (1ull << shift);
+  const uint32_t need_eq = s_remaining;
+  const int nw = blockDim.x >> 5;
+  const int chunk = (((Mo + 31) / 32 + nw - 1) / nw) * 32;
+  const int wb = min(Mo, warp * chunk), we = min(Mo, wb + chunk);
+  auto plain_take = [&](int j, uint32_t rel) -> bool {
+    if (mode == 0) return rel > T;
+    if (mode == 1) return rel >= T;
+    return static_cast<uint64_t>(rel) >= next_floor || ((chosen[j >> 5] >> (j & 31)) & 1u);
+  };
+  uint32_t cnt = 0, cnt_eq = 0;
+  for (int b0 = wb; b0 < we; b0 += 32) {
+    const int j = b0 + lane;
+    const bool in = j < we;
+    const uint32_t rel = in ? key_at(j) - base : 0u;
+    cnt += __popc(__ballot_sync(0xffffffffu, in && plain_take(j, rel)));
+    cnt_eq += __popc(__ballot_sync(0xffffffffu, in && mode == 0 && rel == T));
+  }
+  uint32_t eq_seen = 0;
+  if (mode == 0) eq_seen = warp_exclusive_offset(cnt_eq, warp_tot, &s_total);
+  const uint32_t eq_take = mode == 0
+      ? (eq_seen >= need_eq ? 0u : min(cnt_eq, need_eq - eq_seen)) : 0u;
+  uint32_t pos = warp_exclusive_offset(cnt + eq_take, warp_tot, &s_total);
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int b0 = wb; b0 < we; b0 += 32) {
+    const int j = b0 + lane;
+    const bool in = j < we;
+    const uint32_t rel = in ? key_at(j) - base : 0u;
+    bool take = in && plain_take(j, rel);
+    if (mode == 0) {
+      const uint32_t eqb = __ballot_sync(0xffffffffu, in && rel == T);
+      if (in && rel == T) take = eq_seen + __popc(eqb & lt) < need_eq;
+      eq_seen += __popc(eqb);
+    }
+    const uint32_t tb = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos + __popc(tb & lt)] = j;
+    pos += __popc(tb);
+  }
+  if (tid == 0) out[need] = M - 1;
+}
 
-  const int per = (Mo + blockDim.x - 1) / blockDim.x;
-  const int j0 = min(Mo, tid * per), j1 = min(Mo, j0 + per);
-  uint32_t n_sel = 0, seen = 0, n_eq = 0;
-  if (whole_bin) {
-    for (int j = j0; j < j1; ++j) n_sel += (key_at(j) - base) >= T;
-  } else {
-    for (int j = j0; j < j1; ++j) n_eq += (key_at(j) - base) == T;
-    seen = block_exclusive_scan(n_eq, warp_tot, &s_total);
-    const uint32_t eq_before = seen;
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t rel = key_at(j) - base;
-      if (rel > T) ++n_sel;
-      else if (rel == T) { if (seen < need_eq) ++n_sel; ++seen; }
-    }
-    seen = eq_before;
+// Exclusive scan of a [KPT][32] table of per-(round, warp) counts in
+// (round, warp) order, in place; one warp does it. Returns the total.
+template <int KPT>
+__device__ __forceinline__ uint32_t scan_round_warp_table(uint32_t* tab) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v[KPT], local = 0;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) { v[i] = tab[lane * KPT + i]; local += v[i]; }
+  uint32_t inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
   }
-  uint32_t pos = block_exclusive_scan(n_sel, warp_tot, &s_total);
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t rel = key_at(j) - base;
-    bool take;
-    if (whole_bin) {
-      take = rel >= T;
-    } else {
-      take = rel > T;
-      if (rel == T) { take = seen < need_eq; ++seen; }
+  uint32_t run = inc - local;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) { tab[lane * KPT + i] = run; run += v[i]; }
+  return __shfl_sync(0xffffffffu, inc, 31);
+}
+
+// Selection with every key in registers (M - 1 <= KPT * 1024): thread t holds
+// blocks t, t + 1024, ..., so the index order of the output is (round k,
+// warp, lane). Same result as select_kernel: block M-1 plus the n-1 best of
+// the rest, ties to the lower index, ascending.
+template <int KPT>
+__global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __restrict__ scores,
+                                                                 int32_t* __restrict__ sel, int H,
+                                                                 int M, int n) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t cand_rel[kCand];
+  __shared__ int cand_j[kCand];
+  __shared__ uint32_t chosen[KPT * 32];           // bitmap over block ids (ranked candidates)
+  __shared__ uint32_t tab[KPT * 32];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t red_min[32], red_max[32];
+  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand;
+  __shared__ int s_mode;
+  grid_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
+  const float* s = scores + bh * M;
+  int32_t* out = sel + bh * n;
+  const int Mo = M - 1;
+  const int need = n - 1;
+  if (need >= Mo) {
+    for (int j = tid; j < M; j += blockDim.x) out[j] = j;
+    return;
+  }
+  if (need <= 0) {
+    if (tid == 0) out[0] = M - 1;
+    return;
+  }
+  grid_dependency_wait();                          // scores come from the previous kernel
+  uint32_t kr[KPT];
+  float x[KPT];
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) {
+    const int j = tid + k * kSelThreads;
+    x[k] = j < Mo ? __ldcg(s + j) : 0.f;
+  }
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) {
+    kr[k] = score_key(x[k]);
+    if (tid + k * kSelThreads < Mo) { kmin = min(kmin, kr[k]); kmax = max(kmax, kr[k]); }
+  }
+  for (int b = tid; b < kBins; b += blockDim.x) hist[b] = 0u;
+  if (tid < KPT * 32) chosen[tid] = 0u;
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) { red_min[warp] = kmin; red_max[warp] = kmax; }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = red_min[lane], b = red_max[lane];
+    a = __reduce_min_sync(0xffffffffu, a);
+    b = __reduce_max_sync(0xffffffffu, b);
+    if (lane == 0) {
+      s_kmin = a; s_kmax = b;
+      s_prefix = 0u; s_remaining = static_cast<uint32_t>(need); s_ncand = 0u; s_mode = 0;
     }
-    if (take) out[pos++] = j;
+  }
+  __syncthreads();
+  const uint32_t base = s_kmin;
+  const uint32_t range = s_kmax - base;
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) kr[k] -= base;    // kr now holds rel = key - min
+  auto valid = [&](int k) { return tid + k * kSelThreads < Mo; };
+  int top = 32 - __clz(range);
+  const int shift = top > 11 ? top - 11 : 0;
+  if (top > 0) {
+#pragma unroll
+    for (int k = 0; k < KPT; ++k)
+      if (valid(k)) atomicAdd(&hist[kr[k] >> shift], 1u);
+    __syncthreads();
+    {
+      const uint32_t c0 = hist[kBins - 1 - 2 * tid], c1 = hist[kBins - 2 - 2 * tid];
+      const uint32_t before = block_exclusive_scan(c0 + c1, warp_tot, &s_total);
+      const uint32_t rem = static_cast<uint32_t>(need);
+      uint32_t acc = before;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t c = e == 0 ? c0 : c1;
+        if (acc < rem && rem <= acc + c) {
+          const uint32_t digit = static_cast<uint32_t>(kBins - 1 - 2 * tid - e);
+          s_prefix = digit << shift;
+          s_remaining = rem - acc;
+          s_mode = (rem - acc == c) ? 1 : (c <= static_cast<uint32_t>(kCand) && shift > 0 ? 2 : 0);
+        }
+        acc += c;
+      }
+    }
+    __syncthreads();
+    top = shift;
+    if (s_mode == 2) {
+      const uint32_t bin = s_prefix >> shift;
+#pragma unroll
+      for (int k = 0; k < KPT; ++k) {
+        if (valid(k) && (kr[k] >> shift) == bin) {
+          const uint32_t slot = atomicAdd(&s_ncand, 1u);
+          cand_rel[slot] = kr[k];
+          cand_j[slot] = tid + k * kSelThreads;
+        }
+      }
+      __syncthreads();
+      const int c = static_cast<int>(s_ncand);
+      const uint32_t take = s_remaining;
+      for (int i = tid; i < c; i += blockDim.x) {
+        const uint32_t r = cand_rel[i];
+        const int jj = cand_j[i];
+        uint32_t rank = 0;
+        for (int k = 0; k < c; ++k) {
+          const uint32_t rk = cand_rel[k];
+          rank += (rk > r) || (rk == r && cand_j[k] < jj);
+        }
+        if (rank < take) atomicOr(&chosen[jj >> 5], 1u << (jj & 31));
+      }
+      __syncthreads();
+      top = 0;
+    } else if (s_mode == 1) {
+      top = 0;
+    }
+  }
+  while (top > 0) {                                // crowded threshold bin
+    const int sh = top > 8 ? top - 8 : 0;
+    const int width = top - sh;
+    if (tid < 256) hist[tid] = 0u;
+    __syncthreads();
+    const uint32_t prefix = s_prefix;
+    const uint32_t hi_mask = top >= 32 ? 0u : ~((1u << top) - 1u);
+#pragma unroll
+    for (int k = 0; k < KPT; ++k)
+      if (valid(k) && (kr[k] & hi_mask) == prefix)
+        atomicAdd(&hist[(kr[k] >> sh) & ((1u << width) - 1u)], 1u);
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t c[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * lane - i]; local += c[i]; }
+      uint32_t inc = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const uint32_t before = inc - local;
+      const uint32_t rem = s_remaining;
+      if (before < rem && rem <= inc) {
+        uint32_t acc = before;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (acc < rem && rem <= acc + c[i]) {
+            s_prefix = prefix | (static_cast<uint32_t>(255 - 8 * lane - i) << sh);
+            s_remaining = rem - acc;
+            if (rem - acc == c[i]) s_mode = 1;
+          }
+          acc += c[i];
+        }
+      }
+    }
+    __syncthreads();
+    top = s_mode == 1 ? 0 : sh;
+  }
+  const int mode = s_mode;
+  const uint32_t T = s_prefix;
+  const uint64_t next_floor = static_cast<uint64_t>(T) + (1ull << shift);
+  const uint32_t need_eq = s_remaining;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t take = 0u;                              // bit k: block tid + 1024 k is kept
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) {
+    const uint32_t rel = kr[k];
+    const int j = tid + k * kSelThreads;
+    bool t;
+    if (mode == 0) t = rel > T;
+    else if (mode == 1) t = rel >= T;
+    else t = static_cast<uint64_t>(rel) >= next_floor || ((chosen[j >> 5] >> (j & 31)) & 1u);
+    if (valid(k) && t) take |= 1u << k;
+  }
+  if (mode == 0) {
+    // keys equal to the threshold: the need_eq lowest indices
+#pragma unroll
+    for (int k = 0; k < KPT; ++k) {
+      const uint32_t eqb = __ballot_sync(0xffffffffu, valid(k) && kr[k] == T);
+      if (lane == 0) tab[k * 32 + warp] = __popc(eqb);
+    }
+    __syncthreads();
+    if (warp == 0) scan_round_warp_table<KPT>(tab);
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < KPT; ++k) {
+      const bool eq = valid(k) && kr[k] == T;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      if (eq && tab[k * 32 + warp] + __popc(eqb & lt) < need_eq) take |= 1u << k;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) {
+    const uint32_t tb = __ballot_sync(0xffffffffu, (take >> k) & 1u);
+    if (lane == 0) tab[k * 32 + warp] = __popc(tb);
+  }
+  __syncthreads();
+  if (warp == 0) scan_round_warp_table<KPT>(tab);
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < KPT; ++k) {
+    const bool t = (take >> k) & 1u;
+    const uint32_t tb = __ballot_sync(0xffffffffu, t);
+    if (t) out[tab[k * 32 + warp] + __popc(tb & lt)] = tid + k * kSelThreads;
   }
   if (tid == 0) out[need] = M - 1;
 }
 
 cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int M, int n,
                           cudaStream_t st) {
-  const int in_smem = M <= kSelSmemKeys ? 1 : 0;
-  const size_t smem = in_smem ? static_cast<size_t>(M) * sizeof(uint32_t) : 0;
+  if (M > kSelMaxM) return cudaErrorInvalidValue;
+  const bool in_smem = M <= kSelSmemKeys;
+  const size_t bitmap = static_cast<size_t>((M + 31) / 32) * sizeof(uint32_t);
+  const size_t smem = (in_smem ? static_cast<size_t>(M) * sizeof(uint32_t) : 0) + bitmap;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSelSmemKeys * static_cast<int>(sizeof(uint32_t)));
+    const int most = kSelSmemKeys * static_cast<int>(sizeof(uint32_t)) + (kSelMaxM / 32) * 4;
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               most);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(s.H, s.B);
-  select_kernel<<<grid, kSelThreads, smem, st>>>(scores, sel, s.H, M, n, in_smem);
-  return cudaGetLastError();
+  // programmatic dependent launch: the grid may start while the scores are
+  // still being written; it waits for them on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.H, s.B);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int Mo = M - 1;
+  if (Mo <= 8 * kSelThreads) {
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, select_reg_kernel<8>, scores, sel, s.H, M, n);
+  }
+  if (Mo <= 16 * kSelThreads) {
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, select_reg_kernel<16>, scores, sel, s.H, M, n);
+  }
+  if (in_smem) return cudaLaunchKernelEx(&cfg, select_kernel<true>, scores, sel, s.H, M, n);
+  return cudaLaunchKernelEx(&cfg, select_kernel<false>, scores, sel, s.H, M, n);
 }
 
 }  // namespace resa

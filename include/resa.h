@@ -67,7 +67,8 @@ extern "C" {
 typedef enum {
   RESA_OK = 0,
   RESA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misalignment, len/f/r out of range */
-  RESA_ERR_UNSUPPORTED = -2,  /* head_dim not 64/128, group > 8, block_size != 16 */
+  RESA_ERR_UNSUPPORTED = -2,  /* head_dim not 64/128, group > 8, block_size != 16,
+                                 more than 262144 blocks (4M tokens) to select from */
   RESA_ERR_CAPACITY = -3,     /* len > max_len */
   RESA_ERR_WORKSPACE = -4,    /* workspace smaller than resa_workspace_bytes() */
   RESA_ERR_CUDA = -5,         /* a CUDA runtime/driver call or launch failed */

@@ -114,6 +114,31 @@ def test_all_tied_scores_take_lowest_indices():
         assert np.array_equal(res["gpu_sel"], res["sel"])
 
 
+def test_crowded_ties_take_lowest_indices():
+    """Blocks drawn from three constant patterns: scores take three values, so
+    the threshold is a crowded exact tie broken by block index."""
+    spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=16 * 3000, steps=2,
+                dtype="bf16", r=0.1, n_min=4)
+    K, V = make_cache(spec)
+    rng = np.random.default_rng(99)
+    pats = round_to(rng.standard_normal((3, 128)).astype(np.float32), "bf16")
+    which = rng.integers(0, 3, size=(1, 2, 3000))
+    K[:, :, :spec.len0] = np.repeat(pats[which], 16, axis=2)
+    p = Pair(spec, cache=(K, V))
+    for step in range(spec.steps):
+        res = p.decode(step)
+        assert np.array_equal(res["gpu_sel"], res["sel"])
+
+
+def test_select_beyond_shared_memory_keys():
+    """More blocks than the selection keeps in shared memory (M > 40960)."""
+    spec = Spec(batch=1, n_q_heads=4, n_kv_heads=1, head_dim=64, len0=700_001, steps=2,
+                dtype="bf16", r=0.05, n_min=16)
+    p = Pair(spec)
+    for step in range(spec.steps):
+        p.decode(step)
+
+
 @pytest.mark.parametrize("length,f", [(100, 32), (64, 16), (48, 48), (1000, 7), (1000, 64)])
 def test_rectify_shapes(length, f):
     for dtype in ("bf16", "f32"):
