@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/resa.h"
@@ -122,6 +123,18 @@ int check_dims(const resa_dims* d, Shape* s) {
 }
 
 int64_t blocks_of(int64_t len) { return (len + 15) / 16; }
+
+// The three-kernel decode step (score, select, attend, chained by
+// programmatic dependent launch) is the default. RESA_DECODE_FUSED=1 in the
+// environment selects the one-launch kernel for bf16 (decode_fused.cu); it
+// is exact as well, but its per-CTA redundant selection is slower today.
+bool fused_decode_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("RESA_DECODE_FUSED");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
 
 int splits_for(int units, int64_t min_blocks, int num_sms, const Shape& s) {
   const int target = num_sms * attend_ctas_per_sm(s);
@@ -316,6 +329,32 @@ int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
   int32_t* selp = sel ? sel : reinterpret_cast<int32_t*>(ws + w.sel);
+  if (s.bf16 && fused_decode_enabled()) {
+    // one launch: the CTAs of each KV group score, select and attend together
+    const int num_sms = device_sms();
+    if (num_sms <= 0) return RESA_ERR_CUDA;
+    const int groups = s.B * s.H;
+    int cpg = groups >= num_sms ? 1 : num_sms / groups;
+    if (cpg > kMaxSplits) cpg = kMaxSplits;
+    const int M = static_cast<int>(blocks_of(len));
+    if (cpg > M) cpg = M;
+    while (cpg > 1 && (n + cpg - 1) / cpg > fused_max_share()) --cpg;
+    if (M - 1 <= fused_max_keys(s.D) && (n + cpg - 1) / cpg <= fused_max_share()) {
+      FusedLaunch f{};
+      f.s = s; f.q = q; f.k_new = k_new; f.v_new = v_new; f.k = k_cache; f.v = v_cache;
+      f.desc = desc; f.out = out; f.lse = lse; f.sel = sel;
+      f.scores = reinterpret_cast<float*>(ws + w.scores);
+      f.part_o = reinterpret_cast<float*>(ws + w.part_o);
+      f.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+      f.sync = reinterpret_cast<int*>(ws + w.counters) + static_cast<int64_t>(groups);
+      f.ctrl = reinterpret_cast<Ctrl*>(ws);
+      f.len = len; f.M = M; f.n = n; f.cpg = cpg; f.scale = softmax_scale;
+      CUtensorMap tk, tv;
+      if (!make_cache_map(&tk, k_cache, s) || !make_cache_map(&tv, v_cache, s)) return RESA_ERR_CUDA;
+      f.tm_k = &tk; f.tm_v = &tv;
+      return cuda_status(launch_decode_fused(f, static_cast<cudaStream_t>(stream)));
+    }
+  }
   rc = resa_select_blocks(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, selp,
                           workspace, workspace_bytes, stream);
   if (rc != RESA_OK) return rc;

@@ -57,6 +57,33 @@ struct AttnArgs {
 };
 cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st);
 
+// one-launch decode step (bf16): score, select, attend, merge
+struct FusedLaunch {
+  Shape s;
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  void* k;
+  void* v;
+  void* desc;
+  void* out;
+  float* lse;
+  int32_t* sel;
+  float* scores;
+  float* part_o;
+  float* part_ml;
+  int* sync;              // [B*H][2], zero between calls
+  Ctrl* ctrl;
+  int64_t len;
+  int M, n, cpg;
+  float scale;
+  const CUtensorMap* tm_k;
+  const CUtensorMap* tm_v;
+};
+cudaError_t launch_decode_fused(const FusedLaunch& f, cudaStream_t st);
+int fused_max_keys(int D);
+int fused_max_share();
+
 // rectification attention on tcgen05 (bf16, group size 1, 2, 4 or 8)
 struct RectArgs {
   int B, H, Hq, G, D, f, S, mtiles;

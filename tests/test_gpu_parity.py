@@ -20,7 +20,8 @@ pytestmark = pytest.mark.gpu
 if torch.cuda.is_available():
     import __graft_entry__
     __graft_entry__.build()
-    from tests.pair import Pair, close, to_dev, tdt
+    from tests.pair import Pair, check_selection, close, to_dev, tdt
+    from workload import decode_inputs
 
 
 # ------------------------------------------------------------------ descriptors
@@ -65,6 +66,31 @@ def test_bf16_midsize_run_with_rectify():
         p.decode(step)
         if (step + 1) % spec.f == 0:
             p.rectify()
+    assert p.desc_matches()
+
+
+def test_stage_calls_match_oracle():
+    """resa_select_blocks + resa_attend_blocks (the three-kernel path)."""
+    spec = Spec(batch=2, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=9000, steps=3,
+                dtype="bf16", r=0.1, n_min=16)
+    p = Pair(spec)
+    for step in range(spec.steps):
+        q, kn, vn = decode_inputs(spec, step)
+        p.length += 1
+        n = p.resa.num_selected(p.length, spec.r, spec.n_min)
+        sel = torch.empty(2, 8, n, dtype=torch.int32, device="cuda")
+        out = torch.empty(2, 32, 128, dtype=torch.bfloat16, device="cuda")
+        qd = to_dev(q, "bf16")
+        p.resa.select_blocks(qd, to_dev(kn, "bf16"), to_dev(vn, "bf16"), p.k, p.v, p.desc, p.length,
+                             spec.r, spec.n_min, sel, p.ws)
+        p.resa.attend_blocks(qd, p.k, p.v, p.length, sel, 1.0, out, p.ws)
+        ref = p.st.decode(q, kn, vn, spec.r, spec.n_min, 1.0)
+        gsel = sel.cpu().numpy()
+        exact = all(check_selection(gsel[b, g], ref["scores"][b, g], n)
+                    for b in range(2) for g in range(8))
+        if not exact:
+            ref["out"], _ = p.st.attend_with(q, gsel, 1.0)
+        close(out.float().cpu().numpy(), ref["out"], "bf16", f"staged step {step}")
     assert p.desc_matches()
 
 
@@ -230,3 +256,29 @@ def test_config_256k(r):
 def test_config_64k_batch16(r):
     spec = config(4, r=r, steps=2)
     _run_sampled(spec, steps=2, rect_f=(16, 32, 64) if r == 0.1 else (), rows=[0, 7, 15])
+
+
+def test_one_launch_decode_path():
+    """The one-launch decode kernel (selected by RESA_DECODE_FUSED=1), run in a
+    child process so that the choice does not leak into other tests."""
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, '.');"
+        "from tests.pair import Pair;"
+        "from workload import Spec;"
+        "spec = Spec(batch=2, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=20000, steps=6,"
+        "            dtype='bf16', r=0.1, n_min=16);"
+        "p = Pair(spec);"
+        "[p.decode(s) for s in range(spec.steps)];"
+        "assert p.desc_matches();"
+        "spec2 = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=640, steps=2,"
+        "             dtype='bf16', r=0.1, n_min=4);"
+        "p2 = Pair(spec2); [p2.decode(s) for s in range(2)];"
+        "print('one-launch ok')")
+    import os
+    env = dict(os.environ, RESA_DECODE_FUSED="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and "one-launch ok" in r.stdout, r.stdout + r.stderr
