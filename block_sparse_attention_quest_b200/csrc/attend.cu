@@ -96,9 +96,60 @@ __device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, in
   if (!s_last) return;
   __threadfence();
   // last CTA: each thread merges its (head, channel) outputs over all splits.
-  // The partial outputs and the (m, l) pairs of a chunk of up to 32 splits
-  // are loaded together (one round trip to L2) and folded in with an online
-  // log-sum-exp, so no step waits on another load.
+  constexpr int NT = NW * 32;
+  if (a.G * D <= 2 * NT && a.S <= 32) {
+    // common case (at most two outputs per thread, at most 32 splits): every
+    // partial output and every (m, l) pair is requested before any is used,
+    // so the merge costs one round trip to L2
+    float x[2][32];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int idx = threadIdx.x + it * NT;
+      const int h = idx / D, ch = idx % D;
+      const float* po = a.part_o + (head0 + h) * a.S * D + ch;
+#pragma unroll
+      for (int u = 0; u < 32; ++u)
+        x[it][u] = (idx < a.G * D && u < a.S) ? __ldcg(po + static_cast<int64_t>(u) * D) : 0.f;
+    }
+    float* pml = sm;                                   // [G][S][2]
+    float* w_s = sm + 8 * kMaxSplits * 2;             // [S][8]
+    float* l_h = w_s + kMaxSplits * 8;                // [8]
+    float* m_h = l_h + 8;                             // [8]
+    for (int i = threadIdx.x; i < a.G * a.S * 2; i += NT) pml[i] = __ldcg(a.part_ml + head0 * a.S * 2 + i);
+    __syncthreads();
+    {
+      const int lane = threadIdx.x & 31;
+      for (int h = threadIdx.x >> 5; h < a.G; h += NW) {
+        const float mv = lane < a.S ? pml[(h * a.S + lane) * 2] : -INFINITY;
+        const float lv = lane < a.S ? pml[(h * a.S + lane) * 2 + 1] : 0.f;
+        const float mstar = warp_max_xor(mv, 16, 1);
+        const float w = mv == -INFINITY ? 0.f : exp2f(mv - mstar);
+        if (lane < a.S) w_s[lane * 8 + h] = w;
+        float l = w * lv;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) { l_h[h] = l; m_h[h] = mstar; }
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int idx = threadIdx.x + it * NT;
+      if (idx < a.G * D) {
+        const int h = idx / D, ch = idx % D;
+        float o = 0.f;
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+          if (u < a.S) o = fmaf(w_s[u * 8 + h], x[it][u], o);
+        out[(head0 + h) * D + ch] = Dt<T>::from_f(o / l_h[h]);
+        if (a.lse != nullptr && ch == 0) a.lse[head0 + h] = (m_h[h] + log2f(l_h[h])) * 0.69314718055994531f;
+      }
+    }
+    if (threadIdx.x == 0) *counter = 0;
+    return;
+  }
+  // general case: chunks of up to 32 splits, each loaded in one round trip
+  // and folded in with an online log-sum-exp
   for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
     const int h = idx / D, ch = idx % D;
     const float* po = a.part_o + (head0 + h) * a.S * D + ch;
@@ -239,6 +290,16 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   };
   if (lane == 0) {
     for (int k = 0; k < my_count && k < STAGES; ++k) issue(k);
+  }
+  // the rest of this warp's blocks go to L2 now: the ring above holds only
+  // STAGES tiles per warp, the prefetch keeps the whole share in flight
+  for (int k = STAGES + lane; k < my_count; k += 32) {
+    const int j = block_of(k);
+    if (j >= 0) {
+      const int64_t off = (row_base + static_cast<int64_t>(j) * kBlock) * D;
+      prefetch_l2_bulk(static_cast<const __nv_bfloat16*>(a.k) + off, kBlock * D * 2);
+      prefetch_l2_bulk(static_cast<const __nv_bfloat16*>(a.v) + off, kBlock * D * 2);
+    }
   }
 
   float o[KT][4];
