@@ -34,12 +34,17 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-WORKLOADS = {"32k": 1, "128k": 2, "256k": 3, "64k": 4}
+WORKLOADS = {"tiny": 0, "32k": 1, "128k": 2, "256k": 3, "64k": 4}
 WORKLOAD_NAMES = {
-    1: "resa_decode_32k_b4_needles", 2: "resa_decode_128k_b1", 3: "resa_decode_256k_b1",
+    0: "resa_decode_tiny_fp32", 1: "resa_decode_32k_b4_needles", 2: "resa_decode_128k_b1", 3: "resa_decode_256k_b1",
     4: "resa_decode_64k_b16",
 }
 METRIC = "ReSA decode-step us & achieved HBM GB/s vs roofline at 128K/256K; rectify us"
+
+# DRAM bytes (read + write) per launch of the attention kernel from one ncu
+# capture of this workload (profiles/attend_bf16_kernel_128k.md). Reset an
+# entry to None whenever attend_bf16_kernel changes.
+NCU_TRAFFIC = {"resa_decode_128k_b1": 54220032}
 
 
 def parse():
@@ -112,6 +117,17 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest value over all ranks (timings are reported as the slowest
+    rank's); identity without a process group."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ----------------------------------------------------------------- GPU arm
@@ -269,10 +285,7 @@ def run_ours(args, rank, world, local_rank):
         graph.replay()
         torch.cuda.synchronize()
     clocks = sampler.stop()
-    if dist is not None:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     step_ms = total_ms / args.steps
 
     # per-stage breakdown (graph with captured timing events)
@@ -296,14 +309,33 @@ def run_ours(args, rank, world, local_rank):
                 sel_us.append(e0.elapsed_time(e1) * 1000.0)
                 att_us.append(e1.elapsed_time(e2) * 1000.0)
 
+    # the attention kernel on its own: f * L launches back to back (every
+    # layer's selected blocks, so consecutive launches read different caches)
+    graph_a = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_a, stream=stream):
+        for t in range(f):
+            q = dec_in[t][0]
+            for li, ly in enumerate(layers):
+                resa.attend_blocks(q, ly["k"], ly["v"], len_start + t + 1, sels[li][t], 1.0,
+                                   outs[li], ws[li], lse=lses[li])
+    graph_a.replay()
+    torch.cuda.synchronize()
+    ta0 = torch.cuda.Event(enable_timing=True)
+    ta1 = torch.cuda.Event(enable_timing=True)
+    reps_a = max(3, min(args.steps, 10))
+    with torch.cuda.stream(stream):
+        ta0.record(stream)
+        for _ in range(reps_a):
+            graph_a.replay()
+        ta1.record(stream)
+    torch.cuda.synchronize()
+    attend_launch_us = ta0.elapsed_time(ta1) * 1000.0 / (reps_a * f * L)
+
     # end-to-end through the public API with host buffers (eager calls)
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt)
-        if dist is not None:
-            tt = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(tt.item())
+        e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
 
     assert resa.workspace_status(ws[0]) == resa.RESA_OK
     # bytes of the algorithm (descriptors + selected K/V + Q/O)
@@ -326,7 +358,7 @@ def run_ours(args, rank, world, local_rank):
     decode_med = statistics.median(dec_us)
     staged_med = statistics.median([a + b for a, b in zip(sel_us, att_us)])
     dec_gbs = decode_bytes / (decode_med * 1e-6) / 1e9
-    att_gbs = attend_bytes / (att_med * 1e-6) / 1e9
+    att_gbs = attend_bytes / (attend_launch_us * 1e-6) / 1e9
     us_per_decode = step_ms * 1000.0 / (f * L) / world
     tokens_per_s = B * f * L * world / (step_ms * 1e-3) / L
     launches_per_step = f * L * 3 + L * 3
@@ -357,7 +389,8 @@ def run_ours(args, rank, world, local_rank):
         "staged_decode_us": round(staged_med, 3),
         "staged_select_us": round(sel_med, 3),
         "staged_attend_us": round(att_med, 3),
-        "staged_attend_hbm_gbs": round(att_gbs, 1),
+        "attend_launch_us": round(attend_launch_us, 3),
+        "attend_hbm_gbs": round(att_gbs, 1),
         "decode_hbm_gbs": round(decode_bytes / (decode_med * 1e-6) / 1e9, 1),
         "decode_bytes": decode_bytes,
         "decode_frac_of_measured_hbm": round(decode_bytes / (decode_med * 1e-6) / 1e9 / hbm_peak, 4),
@@ -369,8 +402,10 @@ def run_ours(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_per_s, 1),
         "roofline": {
             "kernel": "attend_bf16_kernel (split-KV attention, LSE merge in the last CTA)",
+            "timing": "average over f * layers back-to-back launches in one CUDA graph",
             "bound": "hbm", "achieved": round(att_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(att_gbs / hbm_peak, 4), "traffic": None,
+            "frac": round(att_gbs / hbm_peak, 4),
+            "traffic": NCU_TRAFFIC.get(WORKLOAD_NAMES[cfg_idx]) if args.r is None else None,
             "peak_kind": f"{peak_kind} copy bandwidth",
             "bytes_per_launch": attend_bytes,
             "bytes": "selected K/V + q + out + block ids",
