@@ -291,16 +291,6 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   if (lane == 0) {
     for (int k = 0; k < my_count && k < STAGES; ++k) issue(k);
   }
-  // the rest of this warp's blocks go to L2 now: the ring above holds only
-  // STAGES tiles per warp, the prefetch keeps the whole share in flight
-  for (int k = STAGES + lane; k < my_count; k += 32) {
-    const int j = block_of(k);
-    if (j >= 0) {
-      const int64_t off = (row_base + static_cast<int64_t>(j) * kBlock) * D;
-      prefetch_l2_bulk(static_cast<const __nv_bfloat16*>(a.k) + off, kBlock * D * 2);
-      prefetch_l2_bulk(static_cast<const __nv_bfloat16*>(a.v) + off, kBlock * D * 2);
-    }
-  }
 
   float o[KT][4];
 #pragma unroll

@@ -536,11 +536,6 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
   if (lane == 0) {
     for (int kx = 0; kx < my_count && kx < kFStages; ++kx) issue(kx);
   }
-  for (int kx = kFStages + lane; kx < my_count; kx += 32) {
-    const int64_t off = (row_base + static_cast<int64_t>(block_of(kx)) * kBlock) * D;
-    prefetch_l2_bulk(a.k + off, kBlock * D * 2);
-    prefetch_l2_bulk(a.v + off, kBlock * D * 2);
-  }
   float o[KT][4];
 #pragma unroll
   for (int mt = 0; mt < KT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
