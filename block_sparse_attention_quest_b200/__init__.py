@@ -40,7 +40,9 @@ BLOCK = 16
 EXPORTED = ("resa_num_selected", "resa_workspace_bytes", "resa_build_desc",
             "resa_decode_sparse", "resa_select_blocks", "resa_attend_blocks",
             "resa_decode_dense", "resa_rectify",
-            "resa_workspace_status", "resa_status_string", "resa_decode_sparse_noalloc")
+            "resa_workspace_status", "resa_status_string", "resa_decode_sparse_noalloc",
+            "resa_build_desc_varlen", "resa_decode_sparse_varlen", "resa_decode_dense_varlen",
+            "resa_rectify_varlen")
 
 
 class Dims(ctypes.Structure):
@@ -77,6 +79,20 @@ _lib.resa_decode_sparse_noalloc.restype = ctypes.c_int
 _lib.resa_decode_sparse_noalloc.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P,
                                             ctypes.c_int64, ctypes.c_double, ctypes.c_int32,
                                             ctypes.c_float, _P, _P, _P, _P]
+_lib.resa_build_desc_varlen.restype = ctypes.c_int
+_lib.resa_build_desc_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, ctypes.c_int64, _P, _P]
+_lib.resa_decode_sparse_varlen.restype = ctypes.c_int
+_lib.resa_decode_sparse_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P,
+                                           ctypes.c_int64, ctypes.c_double, ctypes.c_int32,
+                                           ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.resa_decode_dense_varlen.restype = ctypes.c_int
+_lib.resa_decode_dense_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_int64, ctypes.c_float, _P, _P, _P,
+                                          ctypes.c_size_t, _P]
+_lib.resa_rectify_varlen.restype = ctypes.c_int
+_lib.resa_rectify_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P,
+                                     ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P,
+                                     ctypes.c_size_t, _P]
 _lib.resa_workspace_status.restype = ctypes.c_int
 _lib.resa_workspace_status.argtypes = [_P, _P]
 _lib.resa_status_string.restype = ctypes.c_char_p
@@ -210,3 +226,50 @@ def decode_sparse_noalloc(q, k_new, v_new, k_cache, v_cache, desc, length: int, 
 def workspace_status(workspace, stream=None) -> int:
     """Synchronise and read (and clear) the device error flag of a workspace."""
     return _lib.resa_workspace_status(_ptr(workspace), _stream(stream))
+
+
+# ---- variable-length batches: `lens` is an int32 CUDA tensor [batch] of row
+# lengths, `len_bound` an upper bound on its entries (sizes grids, workspace and
+# the stride of `sel`)
+
+
+def _lens(lens):
+    if lens is None or lens.dtype != torch.int32 or not lens.is_cuda or lens.dim() != 1:
+        raise ValueError("lens must be a 1-D int32 CUDA tensor")
+    return _ptr(lens)
+
+
+def build_desc_varlen(k_cache, lens, len_bound: int, desc, n_q_heads: int, stream=None) -> None:
+    dims = dims_for(k_cache, n_q_heads)
+    _check(_lib.resa_build_desc_varlen(ctypes.byref(dims), _ptr(k_cache), _lens(lens),
+                                       int(len_bound), _ptr(desc), _stream(stream)),
+           "resa_build_desc_varlen")
+
+
+def decode_sparse_varlen(q, k_new, v_new, k_cache, v_cache, desc, lens, len_bound: int, r: float,
+                         n_min: int, softmax_scale: float, out, workspace, lse=None, sel=None,
+                         stream=None) -> None:
+    dims = dims_for(k_cache, q.shape[1])
+    _check(_lib.resa_decode_sparse_varlen(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(desc), _lens(lens), int(len_bound), float(r), int(n_min), float(softmax_scale),
+        _ptr(out), _ptr(lse), _ptr(sel), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "resa_decode_sparse_varlen")
+
+
+def decode_dense_varlen(q, k_new, v_new, k_cache, v_cache, desc, lens, len_bound: int,
+                        softmax_scale: float, out, workspace, lse=None, stream=None) -> None:
+    dims = dims_for(k_cache, q.shape[1])
+    _check(_lib.resa_decode_dense_varlen(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(desc), _lens(lens), int(len_bound), float(softmax_scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel(), _stream(stream)), "resa_decode_dense_varlen")
+
+
+def rectify_varlen(q_f, k_f, v_f, k_cache, v_cache, desc, lens, len_bound: int, f: int,
+                   softmax_scale: float, out_f, workspace, stream=None) -> None:
+    dims = dims_for(k_cache, q_f.shape[2])
+    _check(_lib.resa_rectify_varlen(
+        ctypes.byref(dims), _ptr(q_f), _ptr(k_f), _ptr(v_f), _ptr(k_cache), _ptr(v_cache),
+        _ptr(desc), _lens(lens), int(len_bound), int(f), float(softmax_scale), _ptr(out_f),
+        _ptr(workspace), workspace.numel(), _stream(stream)), "resa_rectify_varlen")

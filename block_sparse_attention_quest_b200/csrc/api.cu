@@ -171,11 +171,16 @@ WsLayout ws_layout(const Shape& s, int64_t len, int32_t f) {
   off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(int32_t));
   // decode rows: B*Hq with units B*H; rectify rows: B*f*Hq with units B*H*f
   const int64_t dec = static_cast<int64_t>(s.B) * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H);
-  const int64_t fr = f > 0 ? f : 1;
-  int64_t sb = split_bound(static_cast<int64_t>(s.B) * s.H * fr);
-  const int64_t sb_tc = split_bound(static_cast<int64_t>(s.B) * s.H * rect_mtiles(s, static_cast<int>(fr)));
-  if (sb_tc > sb) sb = sb_tc;
-  const int64_t rec = static_cast<int64_t>(s.B) * fr * s.Hq * sb;
+  // a smaller window can take more splits, so size for the largest need of
+  // every window up to f
+  int64_t rec = 0;
+  for (int64_t fr = 1; fr <= (f > 0 ? f : 1); ++fr) {
+    int64_t sb = split_bound(static_cast<int64_t>(s.B) * s.H * fr);
+    const int64_t sb_tc = split_bound(static_cast<int64_t>(s.B) * s.H * rect_mtiles(s, static_cast<int>(fr)));
+    if (sb_tc > sb) sb = sb_tc;
+    const int64_t need = static_cast<int64_t>(s.B) * fr * s.Hq * sb;
+    if (need > rec) rec = need;
+  }
   const int64_t rows = dec > rec ? dec : rec;
   w.part_ml = off;
   off = align_up(off + static_cast<size_t>(rows) * 2 * sizeof(float));
@@ -190,7 +195,8 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? RESA_OK : RESA_ERR_CU
 // split-KV attention over `R` query rows + merge
 int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int32_t* sel, int n_sel,
                   float scale, const void* k, const void* v, void* out, float* lse, uint8_t* ws,
-                  const WsLayout& w, int num_sms, cudaStream_t st, bool pdl = false) {
+                  const WsLayout& w, int num_sms, cudaStream_t st, bool pdl = false,
+                  const int32_t* lens = nullptr, double r = 0.0, int n_min = 0) {
   const int64_t min_blocks = sel ? n_sel : blocks_of(len0);
   const int S = splits_for(s.B * s.H * R, min_blocks, num_sms, s);
   AttnArgs a{};
@@ -203,6 +209,7 @@ int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int3
   a.ctrl = reinterpret_cast<Ctrl*>(ws);
   a.k = k; a.v = v;
   a.pdl = pdl;
+  a.lens = lens; a.r = r; a.n_min = n_min;
   CUtensorMap tk, tv;
   if (s.bf16) {
     if (!make_cache_map(&tk, k, s) || !make_cache_map(&tv, v, s)) return RESA_ERR_CUDA;
@@ -235,14 +242,30 @@ size_t resa_workspace_bytes(const resa_dims* dims, int64_t len, int32_t f) {
   return ws_layout(s, len, f).total;
 }
 
-int resa_build_desc(const resa_dims* dims, const void* k_cache, int64_t len, void* desc,
-                    void* stream) {
+static int build_desc_impl(const resa_dims* dims, const void* k_cache, int64_t len, void* desc,
+                           void* stream, const int32_t* lens) {
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != RESA_OK) return rc;
   if (!k_cache || !desc || !aligned16(k_cache) || !aligned16(desc) || len < 1) return RESA_ERR_INVALID_ARG;
   if (len > s.L_max) return RESA_ERR_CAPACITY;
-  return cuda_status(launch_build_desc(s, k_cache, desc, len, static_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_build_desc(s, k_cache, desc, len, static_cast<cudaStream_t>(stream), lens));
+}
+
+int resa_build_desc(const resa_dims* dims, const void* k_cache, int64_t len, void* desc,
+                    void* stream) {
+  return build_desc_impl(dims, k_cache, len, desc, stream, nullptr);
+}
+
+static bool lens_ok(const int32_t* lens) {
+  return lens != nullptr && (reinterpret_cast<uintptr_t>(lens) & 3u) == 0;
+}
+
+int resa_build_desc_varlen(const resa_dims* dims, const void* k_cache, const int32_t* lens,
+                           int64_t len_bound, void* desc, void* stream) {
+  if (!lens_ok(lens)) return RESA_ERR_INVALID_ARG;
+  return build_desc_impl(dims, k_cache, len_bound, desc, stream, lens);
 }
 
 static int check_decode_common(const resa_dims* dims, Shape* s, const void* q, const void* k_new,
@@ -263,10 +286,10 @@ static int check_decode_common(const resa_dims* dims, Shape* s, const void* q, c
   return RESA_OK;
 }
 
-int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
+static int select_impl(const resa_dims* dims, const void* q, const void* k_new,
                        const void* v_new, void* k_cache, void* v_cache, void* desc,
                        int64_t len, double r, int32_t n_min, int32_t* sel, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+                       size_t workspace_bytes, void* stream, const int32_t* lens) {
   Shape s;
   int rc = check_decode_common(dims, &s, q, k_new, v_new, k_cache, v_cache, len, q, workspace,
                                workspace_bytes, 0);
@@ -283,15 +306,24 @@ int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
   const WsLayout w = ws_layout(s, len, 0);
   float* scores = reinterpret_cast<float*>(ws + w.scores);
   cudaError_t e = launch_score(s, q, desc, scores, k_new, v_new, k_cache, v_cache, desc, len,
-                               num_sms, st);
+                               num_sms, st, lens, reinterpret_cast<Ctrl*>(ws));
   if (e != cudaSuccess) return RESA_ERR_CUDA;
-  return cuda_status(launch_select(s, scores, sel, M, n, st));
+  return cuda_status(launch_select(s, scores, sel, M, n, st, lens, len, r, n_min));
+}
+
+int resa_select_blocks(const resa_dims* dims, const void* q, const void* k_new,
+                       const void* v_new, void* k_cache, void* v_cache, void* desc,
+                       int64_t len, double r, int32_t n_min, int32_t* sel, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return select_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, sel,
+                     workspace, workspace_bytes, stream, nullptr);
 }
 
 static int attend_blocks_impl(const resa_dims* dims, const void* q, const void* k_cache,
                               const void* v_cache, int64_t len, const int32_t* sel, int32_t n_sel,
                               float softmax_scale, void* out, float* lse, void* workspace,
-                              size_t workspace_bytes, void* stream, bool pdl) {
+                              size_t workspace_bytes, void* stream, bool pdl,
+                              const int32_t* lens = nullptr, double r = 0.0, int32_t n_min = 0) {
   Shape s;
   int rc = check_decode_common(dims, &s, q, nullptr, nullptr, k_cache, v_cache, len, out,
                                workspace, workspace_bytes, 0);
@@ -303,7 +335,7 @@ static int attend_blocks_impl(const resa_dims* dims, const void* q, const void* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
   return run_attention(s, q, 1, len, sel, n_sel, softmax_scale, k_cache, v_cache, out, lse, ws, w,
-                       num_sms, static_cast<cudaStream_t>(stream), pdl);
+                       num_sms, static_cast<cudaStream_t>(stream), pdl, lens, r, n_min);
 }
 
 int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache,
@@ -314,11 +346,11 @@ int resa_attend_blocks(const resa_dims* dims, const void* q, const void* k_cache
                             workspace, workspace_bytes, stream, false);
 }
 
-int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
-                       const void* v_new, void* k_cache, void* v_cache, void* desc,
-                       int64_t len, double r, int32_t n_min, float softmax_scale, void* out,
-                       float* lse, int32_t* sel, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+static int decode_sparse_impl(const resa_dims* dims, const void* q, const void* k_new,
+                              const void* v_new, void* k_cache, void* v_cache, void* desc,
+                              int64_t len, double r, int32_t n_min, float softmax_scale,
+                              void* out, float* lse, int32_t* sel, void* workspace,
+                              size_t workspace_bytes, void* stream, const int32_t* lens) {
   Shape s;
   int rc = check_decode_common(dims, &s, q, k_new, v_new, k_cache, v_cache, len, out, workspace,
                                workspace_bytes, 0);
@@ -329,7 +361,7 @@ int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
   int32_t* selp = sel ? sel : reinterpret_cast<int32_t*>(ws + w.sel);
-  if (s.bf16 && fused_decode_enabled()) {
+  if (s.bf16 && lens == nullptr && fused_decode_enabled()) {
     // one launch: the CTAs of each KV group score, select and attend together
     const int num_sms = device_sms();
     if (num_sms <= 0) return RESA_ERR_CUDA;
@@ -355,19 +387,41 @@ int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
       return cuda_status(launch_decode_fused(f, static_cast<cudaStream_t>(stream)));
     }
   }
-  rc = resa_select_blocks(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, selp,
-                          workspace, workspace_bytes, stream);
+  rc = select_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, selp,
+                   workspace, workspace_bytes, stream, lens);
   if (rc != RESA_OK) return rc;
   // the attention kernel is a programmatic dependent of the select kernel:
   // its prologue overlaps the selection, it reads the block list after it
   return attend_blocks_impl(dims, q, k_cache, v_cache, len, selp, n, softmax_scale, out, lse,
-                            workspace, workspace_bytes, stream, true);
+                            workspace, workspace_bytes, stream, true, lens, r, n_min);
 }
 
-int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
-                      const void* v_new, void* k_cache, void* v_cache, void* desc, int64_t len,
-                      float softmax_scale, void* out, float* lse, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+int resa_decode_sparse(const resa_dims* dims, const void* q, const void* k_new,
+                       const void* v_new, void* k_cache, void* v_cache, void* desc,
+                       int64_t len, double r, int32_t n_min, float softmax_scale, void* out,
+                       float* lse, int32_t* sel, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  return decode_sparse_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min,
+                            softmax_scale, out, lse, sel, workspace, workspace_bytes, stream,
+                            nullptr);
+}
+
+int resa_decode_sparse_varlen(const resa_dims* dims, const void* q, const void* k_new,
+                              const void* v_new, void* k_cache, void* v_cache, void* desc,
+                              const int32_t* lens, int64_t len_bound, double r, int32_t n_min,
+                              float softmax_scale, void* out, float* lse, int32_t* sel,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!lens_ok(lens)) return RESA_ERR_INVALID_ARG;
+  return decode_sparse_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len_bound, r, n_min,
+                            softmax_scale, out, lse, sel, workspace, workspace_bytes, stream,
+                            lens);
+}
+
+static int decode_dense_impl(const resa_dims* dims, const void* q, const void* k_new,
+                             const void* v_new, void* k_cache, void* v_cache, void* desc,
+                             int64_t len, float softmax_scale, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream,
+                             const int32_t* lens) {
   Shape s;
   int rc = check_decode_common(dims, &s, q, k_new, v_new, k_cache, v_cache, len, out, workspace,
                                workspace_bytes, 0);
@@ -380,17 +434,35 @@ int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
   if (k_new) {
-    cudaError_t e = launch_append(s, k_new, v_new, k_cache, v_cache, desc, len, st);
+    cudaError_t e = launch_append(s, k_new, v_new, k_cache, v_cache, desc, len, st, lens);
     if (e != cudaSuccess) return RESA_ERR_CUDA;
   }
   return run_attention(s, q, 1, len, nullptr, 0, softmax_scale, k_cache, v_cache, out, lse, ws, w,
-                       num_sms, st);
+                       num_sms, st, false, lens);
 }
 
-int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
-                 void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
-                 float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
-                 void* stream) {
+int resa_decode_dense(const resa_dims* dims, const void* q, const void* k_new,
+                      const void* v_new, void* k_cache, void* v_cache, void* desc, int64_t len,
+                      float softmax_scale, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  return decode_dense_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len, softmax_scale, out,
+                           lse, workspace, workspace_bytes, stream, nullptr);
+}
+
+int resa_decode_dense_varlen(const resa_dims* dims, const void* q, const void* k_new,
+                             const void* v_new, void* k_cache, void* v_cache, void* desc,
+                             const int32_t* lens, int64_t len_bound, float softmax_scale,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (!lens_ok(lens)) return RESA_ERR_INVALID_ARG;
+  return decode_dense_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len_bound,
+                           softmax_scale, out, lse, workspace, workspace_bytes, stream, lens);
+}
+
+static int rectify_impl(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
+                        void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
+                        float softmax_scale, void* out_f, void* workspace,
+                        size_t workspace_bytes, void* stream, const int32_t* lens) {
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != RESA_OK) return rc;
@@ -405,7 +477,8 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, f);
-  cudaError_t e = launch_rectify_write(s, k_f, v_f, k_cache, v_cache, desc, len, f, st);
+  cudaError_t e = launch_rectify_write(s, k_f, v_f, k_cache, v_cache, desc, len, f, st, lens,
+                                       reinterpret_cast<Ctrl*>(ws));
   if (e != cudaSuccess) return RESA_ERR_CUDA;
   if (rectify_on_tensor_cores(s)) {
     RectArgs r{};
@@ -417,7 +490,7 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
     if (S > kMaxSplits) S = kMaxSplits;
     if (S > n_tiles) S = n_tiles;
     r.S = static_cast<int>(S);
-    r.len = len; r.L_max = s.L_max; r.scale = softmax_scale; r.out = out_f;
+    r.len = len; r.lens = lens; r.L_max = s.L_max; r.scale = softmax_scale; r.out = out_f;
     r.part_o = reinterpret_cast<float*>(ws + w.part_o);
     r.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
     r.ctrl = reinterpret_cast<Ctrl*>(ws);
@@ -429,7 +502,24 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
     return cuda_status(launch_rectify_tc(r, st));
   }
   return run_attention(s, q_f, f, len - f + 1, nullptr, 0, softmax_scale, k_cache, v_cache, out_f,
-                       nullptr, ws, w, num_sms, st);
+                       nullptr, ws, w, num_sms, st, false, lens);
+}
+
+int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
+                 void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
+                 float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  return rectify_impl(dims, q_f, k_f, v_f, k_cache, v_cache, desc, len, f, softmax_scale, out_f,
+                      workspace, workspace_bytes, stream, nullptr);
+}
+
+int resa_rectify_varlen(const resa_dims* dims, const void* q_f, const void* k_f,
+                        const void* v_f, void* k_cache, void* v_cache, void* desc,
+                        const int32_t* lens, int64_t len_bound, int32_t f, float softmax_scale,
+                        void* out_f, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!lens_ok(lens)) return RESA_ERR_INVALID_ARG;
+  return rectify_impl(dims, q_f, k_f, v_f, k_cache, v_cache, desc, len_bound, f, softmax_scale,
+                      out_f, workspace, workspace_bytes, stream, lens);
 }
 
 int resa_workspace_status(void* workspace, void* stream) {
@@ -457,7 +547,7 @@ const char* resa_status_string(int status) {
     case RESA_ERR_WORKSPACE: return "workspace too small";
     case RESA_ERR_CUDA: return "CUDA error";
     case RESA_ERR_TIMEOUT: return "device-side wait timed out";
-    case RESA_ERR_BAD_INDEX: return "block id out of range in the selection";
+    case RESA_ERR_BAD_INDEX: return "block id or per-row length out of range";
     default: return "unknown status";
   }
 }

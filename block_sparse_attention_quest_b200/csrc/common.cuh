@@ -13,7 +13,7 @@ namespace resa {
 constexpr int kBlock = 16;             // tokens per block (b)
 constexpr int kCtrlBytes = 256;        // workspace control block
 constexpr int kErrTimeout = 1;         // bits of the control block's error word
-constexpr int kErrBadIndex = 2;
+constexpr int kErrBadIndex = 2;        // a block id or a per-row length out of range
 // A device wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -30,6 +30,28 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 
 __device__ __forceinline__ void raise_error(Ctrl* ctrl, int bit) {
   if (ctrl) atomicOr(&ctrl->error, bit);
+}
+
+// ---------------------------------------------------------------- per-row lengths
+// Length of batch row b: lens[b] when a per-row array is given (clamped to
+// [1, bound]), else the shared scalar.
+__device__ __forceinline__ int64_t row_len(const int32_t* lens, int64_t len, int b) {
+  if (lens == nullptr) return len;
+  int64_t l = lens[b];
+  return l < 1 ? 1 : (l > len ? len : l);
+}
+// lens[b] outside [1, bound] (reported once by the first kernel of a call)
+__device__ __forceinline__ bool row_len_bad(const int32_t* lens, int64_t len, int b) {
+  return lens != nullptr && (lens[b] < 1 || static_cast<int64_t>(lens[b]) > len);
+}
+// Block budget of Eq. 5 on the device; the same double-precision formula as
+// resa_num_selected: n = min(M, max(n_min, ceil(M r - 1e-9))).
+__device__ __forceinline__ int num_selected_dev(int64_t len, double r, int n_min) {
+  const int64_t M = (len + kBlock - 1) / kBlock;
+  int64_t n = static_cast<int64_t>(ceil(static_cast<double>(M) * r - 1e-9));
+  if (n < n_min) n = n_min;
+  if (n > M) n = M;
+  return static_cast<int>(n);
 }
 
 // ---------------------------------------------------------------- dtypes
@@ -140,12 +162,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
-}
-// Bulk prefetch of [p, p + bytes) into L2 (fire and forget; 16-byte aligned,
-// size a multiple of 16). Lets a CTA put far more bytes in flight than its
-// registers or shared-memory stages hold.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -19,7 +19,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) build_desc_kernel(const T* __restrict__ k,
                                                          T* __restrict__ desc, int64_t L_max,
                                                          int Mmax, int M, int64_t len,
-                                                         int64_t total) {
+                                                         int64_t total, const int32_t* lens,
+                                                         int H) {
   constexpr int CH = Chunk<T>::N;
   constexpr int CPR = D / CH;                 // 16-byte chunks per token row
   constexpr int TPP = 32 / CPR;               // rows covered by one warp-wide load
@@ -28,7 +29,9 @@ __global__ void __launch_bounds__(256) build_desc_kernel(const T* __restrict__ k
   if (wid >= total) return;
   const int64_t bh = wid / M;
   const int j = static_cast<int>(wid % M);
-  const int valid = static_cast<int>(len - static_cast<int64_t>(j) * kBlock < kBlock ? len - static_cast<int64_t>(j) * kBlock : kBlock);
+  const int64_t len_b = row_len(lens, len, static_cast<int>(bh / H));
+  if (static_cast<int64_t>(j) * kBlock >= len_b) return;     // past this row's length
+  const int valid = static_cast<int>(len_b - static_cast<int64_t>(j) * kBlock < kBlock ? len_b - static_cast<int64_t>(j) * kBlock : kBlock);
   const int chunk = lane % CPR;
   const int r0 = lane / CPR;
   const T* base = k + (bh * L_max + static_cast<int64_t>(j) * kBlock) * D + chunk * CH;
@@ -72,10 +75,10 @@ __global__ void __launch_bounds__(256) build_desc_kernel(const T* __restrict__ k
 template <typename T>
 __global__ void append_kernel(const T* __restrict__ k_new, const T* __restrict__ v_new,
                               T* __restrict__ k, T* __restrict__ v, T* __restrict__ desc, int H,
-                              int D, int64_t L_max, int Mmax, int64_t len) {
+                              int D, int64_t L_max, int Mmax, int64_t len, const int32_t* lens) {
   const int c = threadIdx.x;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
-  const int64_t t = len - 1;
+  const int64_t t = row_len(lens, len, blockIdx.y) - 1;
   const T kn = k_new[bh * D + c];
   k[(bh * L_max + t) * D + c] = kn;
   v[(bh * L_max + t) * D + c] = v_new[bh * D + c];
@@ -98,12 +101,17 @@ __global__ void append_kernel(const T* __restrict__ k_new, const T* __restrict__
 template <typename T>
 __global__ void rectify_write_kernel(const T* __restrict__ k_f, const T* __restrict__ v_f,
                                      T* __restrict__ k, T* __restrict__ v, T* __restrict__ desc,
-                                     int H, int D, int64_t L_max, int Mmax, int64_t len, int f) {
+                                     int H, int D, int64_t L_max, int Mmax, int64_t len, int f,
+                                     const int32_t* lens, Ctrl* ctrl) {
   const int c = threadIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * H + h;
+  if (blockIdx.x == 0 && h == 0 && c == 0 && row_len_bad(lens, len, b)) raise_error(ctrl, kErrBadIndex);
+  len = row_len(lens, len, b);
+  if (len < f) return;                     // a row shorter than the window is left alone
   const int64_t t_first = len - f;
   const int64_t j = t_first / kBlock + blockIdx.x;
+  if (j * kBlock >= len) return;           // this row touches fewer blocks
   const int64_t t0 = j * kBlock;
   const int64_t t1 = t0 + kBlock < len ? t0 + kBlock : len;
   float mn = INFINITY, mx = -INFINITY;
@@ -129,58 +137,62 @@ __global__ void rectify_write_kernel(const T* __restrict__ k_f, const T* __restr
 
 template <typename T, int D>
 static cudaError_t build_desc_t(const Shape& s, const void* k, void* desc, int64_t len,
-                                cudaStream_t st) {
+                                cudaStream_t st, const int32_t* lens) {
   const int M = static_cast<int>((len + kBlock - 1) / kBlock);
   const int64_t total = static_cast<int64_t>(s.B) * s.H * M;
   const int threads = 256;
   const int64_t grid = (total * 32 + threads - 1) / threads;
   build_desc_kernel<T, D><<<static_cast<unsigned>(grid), threads, 0, st>>>(
-      static_cast<const T*>(k), static_cast<T*>(desc), s.L_max, s.Mmax, M, len, total);
+      static_cast<const T*>(k), static_cast<T*>(desc), s.L_max, s.Mmax, M, len, total, lens, s.H);
   return cudaGetLastError();
 }
 
 cudaError_t launch_build_desc(const Shape& s, const void* k, void* desc, int64_t len,
-                              cudaStream_t st) {
+                              cudaStream_t st, const int32_t* lens) {
   if (s.bf16) {
-    return s.D == 128 ? build_desc_t<__nv_bfloat16, 128>(s, k, desc, len, st)
-                      : build_desc_t<__nv_bfloat16, 64>(s, k, desc, len, st);
+    return s.D == 128 ? build_desc_t<__nv_bfloat16, 128>(s, k, desc, len, st, lens)
+                      : build_desc_t<__nv_bfloat16, 64>(s, k, desc, len, st, lens);
   }
-  return s.D == 128 ? build_desc_t<float, 128>(s, k, desc, len, st)
-                    : build_desc_t<float, 64>(s, k, desc, len, st);
+  return s.D == 128 ? build_desc_t<float, 128>(s, k, desc, len, st, lens)
+                    : build_desc_t<float, 64>(s, k, desc, len, st, lens);
 }
 
 cudaError_t launch_append(const Shape& s, const void* k_new, const void* v_new, void* k, void* v,
-                          void* desc, int64_t len, cudaStream_t st) {
+                          void* desc, int64_t len, cudaStream_t st, const int32_t* lens) {
   dim3 grid(s.H, s.B);
   if (s.bf16) {
     using T = __nv_bfloat16;
     append_kernel<T><<<grid, s.D, 0, st>>>(static_cast<const T*>(k_new),
                                            static_cast<const T*>(v_new), static_cast<T*>(k),
                                            static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D,
-                                           s.L_max, s.Mmax, len);
+                                           s.L_max, s.Mmax, len, lens);
   } else {
     append_kernel<float><<<grid, s.D, 0, st>>>(
         static_cast<const float*>(k_new), static_cast<const float*>(v_new),
         static_cast<float*>(k), static_cast<float*>(v), static_cast<float*>(desc), s.H, s.D,
-        s.L_max, s.Mmax, len);
+        s.L_max, s.Mmax, len, lens);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_f, void* k, void* v,
-                                 void* desc, int64_t len, int f, cudaStream_t st) {
+                                 void* desc, int64_t len, int f, cudaStream_t st,
+                                 const int32_t* lens, Ctrl* ctrl) {
+  // blocks touched by f slots: at most f/16 + 2 (the bound covers every row)
   const int64_t j0 = (len - f) / kBlock;
   const int64_t M = (len + kBlock - 1) / kBlock;
-  dim3 grid(static_cast<unsigned>(M - j0), s.H, s.B);
+  const int64_t touched = lens ? f / kBlock + 2 : M - j0;
+  dim3 grid(static_cast<unsigned>(touched), s.H, s.B);
   if (s.bf16) {
     using T = __nv_bfloat16;
     rectify_write_kernel<T><<<grid, s.D, 0, st>>>(
         static_cast<const T*>(k_f), static_cast<const T*>(v_f), static_cast<T*>(k),
-        static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f);
+        static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f, lens, ctrl);
   } else {
     rectify_write_kernel<float><<<grid, s.D, 0, st>>>(
         static_cast<const float*>(k_f), static_cast<const float*>(v_f), static_cast<float*>(k),
-        static_cast<float*>(v), static_cast<float*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f);
+        static_cast<float*>(v), static_cast<float*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f, lens,
+        ctrl);
   }
   return cudaGetLastError();
 }

@@ -18,21 +18,26 @@ struct Shape {
 };
 
 // descriptors ----------------------------------------------------------------
+// lens: optional per-row lengths [B] on the device (len is then their bound)
 cudaError_t launch_build_desc(const Shape& s, const void* k, void* desc, int64_t len,
-                              cudaStream_t st);
+                              cudaStream_t st, const int32_t* lens = nullptr);
 cudaError_t launch_append(const Shape& s, const void* k_new, const void* v_new, void* k, void* v,
-                          void* desc, int64_t len, cudaStream_t st);
+                          void* desc, int64_t len, cudaStream_t st, const int32_t* lens = nullptr);
 cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_f, void* k, void* v,
-                                 void* desc, int64_t len, int f, cudaStream_t st);
+                                 void* desc, int64_t len, int f, cudaStream_t st,
+                                 const int32_t* lens = nullptr, Ctrl* ctrl = nullptr);
 
 // scoring + selection ----------------------------------------------------------
 // scores: [B][H][M] float; the CTA that owns the last chunk also performs the
 // append of (k_new, v_new) when k_new != nullptr.
 cudaError_t launch_score(const Shape& s, const void* q, const void* desc, float* scores,
                          const void* k_new, const void* v_new, void* k, void* v, void* desc_w,
-                         int64_t len, int num_sms, cudaStream_t st);
+                         int64_t len, int num_sms, cudaStream_t st,
+                         const int32_t* lens = nullptr, Ctrl* ctrl = nullptr);
+// with lens, each row's M and n follow its own length (r, n_min: Eq. 5)
 cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int M, int n,
-                          cudaStream_t st);
+                          cudaStream_t st, const int32_t* lens = nullptr, int64_t len = 0,
+                          double r = 0.0, int n_min = 0);
 
 // attention ---------------------------------------------------------------------
 struct AttnArgs {
@@ -54,6 +59,13 @@ struct AttnArgs {
   const void* k;          // cache base pointers (fp32 path)
   const void* v;
   bool pdl;               // launched as a programmatic dependent of the select kernel
+  // optional per-row lengths [B]: row b's last query row sees lens[b] tokens
+  // (len0 + R - 1 is then their bound); a batch row shorter than R is
+  // skipped; selected rows hold Eq. 5's n for their own length (r, n_min),
+  // n_sel being the list stride
+  const int32_t* lens;
+  double r;
+  int n_min;
 };
 cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st);
 
@@ -87,7 +99,8 @@ int fused_max_share();
 // rectification attention on tcgen05 (bf16, group size 1, 2, 4 or 8)
 struct RectArgs {
   int B, H, Hq, G, D, f, S, mtiles;
-  int64_t len, L_max;
+  int64_t len, L_max;     // len: the cache length (with lens: the bound on the rows')
+  const int32_t* lens;    // optional per-row lengths [B]; rows shorter than f are skipped
   float scale;
   void* out;              // [B][f][Hq][D] bf16
   float* part_o;          // [B*f*Hq][S][D]

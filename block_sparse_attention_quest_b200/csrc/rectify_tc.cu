@@ -39,6 +39,7 @@ struct RectK {
   Ctrl* ctrl;
   int64_t len;
   int64_t L_max;
+  const int32_t* lens;   // optional per-row lengths [B] (len: their bound)
   int H, Hq, G, f, S, mtiles;
   float scale_log2;
 };
@@ -86,7 +87,8 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   const int s_idx = blockIdx.x, g = blockIdx.y;
   const int b = blockIdx.z / a.mtiles, mt = blockIdx.z % a.mtiles;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t len = a.len;
+  const int64_t len = row_len(a.lens, a.len, b);
+  if (len < a.f) return;                   // a row shorter than the window is skipped
   const int n_tiles = static_cast<int>((len + 127) / 128);
   const int t0 = static_cast<int>(static_cast<int64_t>(s_idx) * n_tiles / a.S);
   const int t1 = static_cast<int>(static_cast<int64_t>(s_idx + 1) * n_tiles / a.S);
@@ -380,11 +382,14 @@ template <int D>
 __global__ void __launch_bounds__(128) merge_rows_kernel(const float* __restrict__ part_o,
                                                          const float* __restrict__ part_ml,
                                                          __nv_bfloat16* __restrict__ out,
-                                                         int64_t rows, int S) {
+                                                         int64_t rows, int S,
+                                                         const int32_t* lens, int64_t len,
+                                                         int64_t rows_per_b, int f) {
   constexpr int CPL = D / 32;
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
+  if (lens != nullptr && row_len(lens, len, static_cast<int>(row / rows_per_b)) < f) return;
   const float* ml = part_ml + row * S * 2;
   float mstar = -INFINITY;
   for (int s = lane; s < S; s += 32) mstar = fmaxf(mstar, ml[2 * s]);
@@ -443,6 +448,7 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   RectK k{};
   k.out = r.out; k.part_o = r.part_o; k.part_ml = r.part_ml; k.ctrl = r.ctrl;
   k.len = r.len; k.L_max = r.L_max; k.H = r.H; k.Hq = r.Hq; k.G = r.G; k.f = r.f; k.S = r.S;
+  k.lens = r.lens;
   k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
   dim3 grid(r.S, r.H, r.B * r.mtiles);
   rectify_tc_kernel<D><<<grid, 288, C::kSmem, st>>>(*r.tm_q, *r.tm_k, *r.tm_v, k);
@@ -450,7 +456,8 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   if (e != cudaSuccess || r.S == 1) return e;
   const int64_t rows = static_cast<int64_t>(r.B) * r.f * r.Hq;
   merge_rows_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(
-      r.part_o, r.part_ml, static_cast<__nv_bfloat16*>(r.out), rows, r.S);
+      r.part_o, r.part_ml, static_cast<__nv_bfloat16*>(r.out), rows, r.S, r.lens, r.len,
+      static_cast<int64_t>(r.f) * r.Hq, r.f);
   return cudaGetLastError();
 }
 

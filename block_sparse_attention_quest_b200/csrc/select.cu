@@ -73,8 +73,10 @@ struct ScoreArgs {
   void* v;
   void* desc_w;
   int64_t L_max;
-  int64_t len;
-  int H, G, Mmax, M;
+  int64_t len;                // cache length (with lens: the bound on every row's)
+  const int32_t* lens;        // optional per-row lengths [B]
+  Ctrl* ctrl;
+  int H, G, Mmax, M;          // M: blocks of len, the row stride of scores
   int blocks_per_cta;
 };
 
@@ -96,7 +98,10 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(b) * a.H + g;
-  const int last_scored = a.M - 1;                 // block M-1 is forced, not scored
+  const int64_t len_b = row_len(a.lens, a.len, b);
+  if (a.lens != nullptr && blockIdx.x == 0 && g == 0 && tid == 0 && row_len_bad(a.lens, a.len, b))
+    raise_error(a.ctrl, kErrBadIndex);
+  const int last_scored = static_cast<int>((len_b + kBlock - 1) / kBlock) - 1;  // block M-1 is forced, not scored
   const int j_begin = blockIdx.x * a.blocks_per_cta;
   const int j_end = min(j_begin + a.blocks_per_cta, last_scored);
   const T* dbase = static_cast<const T*>(a.desc) + bh * a.Mmax * 2 * D;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
 
   // fused append of the decode token (the scoring above never reads block M-1)
   if (a.k_new != nullptr && blockIdx.x == gridDim.x - 1 && tid < D) {
-    const int64_t t = a.len - 1;
+    const int64_t t = len_b - 1;
     const T kn = static_cast<const T*>(a.k_new)[bh * D + tid];
     static_cast<T*>(a.k)[(bh * a.L_max + t) * D + tid] = kn;
     static_cast<T*>(a.v)[(bh * a.L_max + t) * D + tid] =
@@ -219,8 +224,10 @@ static cudaError_t score_t(const Shape& s, const ScoreArgs& a0, int num_sms, cud
 
 cudaError_t launch_score(const Shape& s, const void* q, const void* desc, float* scores,
                          const void* k_new, const void* v_new, void* k, void* v, void* desc_w,
-                         int64_t len, int num_sms, cudaStream_t st) {
+                         int64_t len, int num_sms, cudaStream_t st, const int32_t* lens,
+                         Ctrl* ctrl) {
   ScoreArgs a{};
+  a.lens = lens; a.ctrl = ctrl;
   a.q = q; a.desc = desc; a.scores = scores; a.k_new = k_new; a.v_new = v_new;
   a.k = k; a.v = v; a.desc_w = desc_w; a.L_max = s.L_max; a.len = len;
   a.H = s.H; a.G = s.G; a.Mmax = s.Mmax;
@@ -303,6 +310,24 @@ __device__ __forceinline__ uint32_t warp_exclusive_offset(uint32_t x, uint32_t* 
   return r;
 }
 
+// Per-row budget for variable lengths: the row's own block count M and
+// Eq. 5 budget n (both at most the shared ones); the list keeps the shared
+// stride and its unused tail is set to -1.
+struct SelRows {
+  const int32_t* lens;   // nullptr: every row has the shared length
+  int64_t len;           // bound on the row lengths
+  double r;
+  int n_min;
+};
+
+__device__ __forceinline__ void row_budget(const SelRows& rl, int b, int& M, int& n, int32_t* out) {
+  const int stride = n;
+  const int64_t lb = row_len(rl.lens, rl.len, b);
+  M = static_cast<int>((lb + kBlock - 1) / kBlock);
+  n = num_selected_dev(lb, rl.r, rl.n_min);
+  for (int i = n + static_cast<int>(threadIdx.x); i < stride; i += blockDim.x) out[i] = -1;
+}
+
 // Grid (H, B). Keeps block M-1 and the n-1 best of blocks 0 .. M-2; among
 // equal scores the lower index wins. Output ascending.
 //
@@ -318,7 +343,7 @@ __device__ __forceinline__ uint32_t warp_exclusive_offset(uint32_t x, uint32_t* 
 template <bool IN_SMEM>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores,
                                                              int32_t* __restrict__ sel, int H,
-                                                             int M, int n) {
+                                                             int M, int n, SelRows rl) {
   extern __shared__ uint32_t dyn[];               // [keys (if in smem)][chosen bitmap]
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t cand_rel[kCand];
@@ -332,6 +357,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
   const float* s = scores + bh * M;
   int32_t* out = sel + bh * n;
+  if (rl.lens != nullptr) row_budget(rl, blockIdx.y, M, n, out);
   const int Mo = M - 1;                            // candidates: blocks 0 .. M-2
   const int need = n - 1;                          // how many of them to keep
   uint32_t* skeys = dyn;
@@ -562,7 +588,7 @@ __device__ __forceinline__ uint32_t scan_round_warp_table(uint32_t* tab) {
 template <int KPT>
 __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __restrict__ scores,
                                                                  int32_t* __restrict__ sel, int H,
-                                                                 int M, int n) {
+                                                                 int M, int n, SelRows rl) {
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t cand_rel[kCand];
   __shared__ int cand_j[kCand];
@@ -577,6 +603,7 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
   const float* s = scores + bh * M;
   int32_t* out = sel + bh * n;
+  if (rl.lens != nullptr) row_budget(rl, blockIdx.y, M, n, out);
   const int Mo = M - 1;
   const int need = n - 1;
   if (need >= Mo) {
@@ -769,7 +796,9 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
 }
 
 cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int M, int n,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int32_t* lens, int64_t len, double r,
+                          int n_min) {
+  const SelRows rl{lens, len, r, n_min};
   if (M > kSelMaxM) return cudaErrorInvalidValue;
   const bool in_smem = M <= kSelSmemKeys;
   const size_t bitmap = static_cast<size_t>((M + 31) / 32) * sizeof(uint32_t);
@@ -802,14 +831,14 @@ cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int
   const int Mo = M - 1;
   if (Mo <= 8 * kSelThreads) {
     cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, select_reg_kernel<8>, scores, sel, s.H, M, n);
+    return cudaLaunchKernelEx(&cfg, select_reg_kernel<8>, scores, sel, s.H, M, n, rl);
   }
   if (Mo <= 16 * kSelThreads) {
     cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, select_reg_kernel<16>, scores, sel, s.H, M, n);
+    return cudaLaunchKernelEx(&cfg, select_reg_kernel<16>, scores, sel, s.H, M, n, rl);
   }
-  if (in_smem) return cudaLaunchKernelEx(&cfg, select_kernel<true>, scores, sel, s.H, M, n);
-  return cudaLaunchKernelEx(&cfg, select_kernel<false>, scores, sel, s.H, M, n);
+  if (in_smem) return cudaLaunchKernelEx(&cfg, select_kernel<true>, scores, sel, s.H, M, n, rl);
+  return cudaLaunchKernelEx(&cfg, select_kernel<false>, scores, sel, s.H, M, n, rl);
 }
 
 }  // namespace resa

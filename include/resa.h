@@ -32,7 +32,8 @@
  *       sel               [batch][n_kv_heads][n]        int32, ascending
  *   - Query head h reads KV head h / (n_q_heads / n_kv_heads).
  *   - `len` is the number of valid tokens in the cache, counting the token a
- *     decode call appends. All batch rows share one len.
+ *     decode call appends. All batch rows share one len, except in the
+ *     *_varlen calls, where row b has lens[b] tokens (see below).
  *   - q, k, v, desc and out share the dtype in resa_dims.dtype; softmax and
  *     accumulation are float32; softmax_scale must be finite and positive.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
@@ -73,7 +74,8 @@ typedef enum {
   RESA_ERR_WORKSPACE = -4,    /* workspace smaller than resa_workspace_bytes() */
   RESA_ERR_CUDA = -5,         /* a CUDA runtime/driver call or launch failed */
   RESA_ERR_TIMEOUT = -6,      /* a device-side wait gave up (flag in the workspace) */
-  RESA_ERR_BAD_INDEX = -7     /* a block id in `sel` was out of range (flag in the workspace) */
+  RESA_ERR_BAD_INDEX = -7     /* a block id in `sel`, or an entry of `lens`, was out of
+                                 range (flag in the workspace) */
 } resa_status;
 
 typedef enum { RESA_F32 = 0, RESA_BF16 = 1 } resa_dtype;
@@ -95,8 +97,9 @@ typedef struct {
 RESA_API int32_t resa_num_selected(int64_t len, int32_t block_size, double r, int32_t n_min);
 
 /* Workspace bytes that suffice for resa_decode_sparse, resa_decode_dense and
- * resa_rectify (with this f) at any length up to `len`. Returns 0 for invalid
- * dims. */
+ * resa_rectify (with any window f' <= f) at any length up to `len`, and for
+ * the *_varlen calls with len_bound <= len. Returns 0 for invalid dims, len < 1
+ * or f outside [0, 256]. */
 RESA_API size_t resa_workspace_bytes(const resa_dims* dims, int64_t len, int32_t f);
 
 /* Quest block descriptors of the first `len` tokens (per-block, per-channel
@@ -195,6 +198,56 @@ RESA_API int resa_decode_sparse_noalloc(const resa_dims* dims, const void* q, co
                                         void* desc, int64_t len, double r, int32_t n_min,
                                         float softmax_scale, void* out, float* lse,
                                         int32_t* sel, void* stream);
+
+/* ---- variable-length batches (continuous batching) ----
+ * The pages run ReSA one sequence at a time; batching sequences of different
+ * lengths is this library's extension and changes nothing per row: every row
+ * computes exactly what the fixed-length call computes at its own length.
+ *  - lens: DEVICE int32 array [batch], 4-byte aligned, owned by the caller;
+ *    lens[b] is row b's token count (counting a decode call's appended token).
+ *  - len_bound >= every lens[b] (for instance the longest row); it sizes the
+ *    grids, the workspace (resa_workspace_bytes(dims, len_bound, f)) and the
+ *    stride n_cap = resa_num_selected(len_bound, 16, r, n_min) of `sel`.
+ *    Host checks apply to len_bound as to len (1 <= len_bound <= max_len).
+ *  - An entry outside [1, len_bound] is clamped into it and raises the
+ *    RESA_ERR_BAD_INDEX flag read by resa_workspace_status() (no flag for
+ *    resa_build_desc_varlen, which has no workspace).
+ *  - lens is read on the device only: the calls can be captured in a CUDA
+ *    graph once and replayed while the lengths change. */
+
+/* resa_build_desc for every row b over its first lens[b] tokens. */
+RESA_API int resa_build_desc_varlen(const resa_dims* dims, const void* k_cache,
+                                    const int32_t* lens, int64_t len_bound, void* desc,
+                                    void* stream);
+
+/* resa_decode_sparse with row b at length lens[b]: the appended token goes to
+ * slot lens[b]-1, row b's KV groups select n_b = resa_num_selected(lens[b],
+ * 16, r, n_min) of its ceil(lens[b]/16) blocks. sel (optional) is
+ * [batch][n_kv_heads][n_cap]: n_b ascending ids, then -1 up to n_cap.
+ * Always runs the three-kernel path. */
+RESA_API int resa_decode_sparse_varlen(const resa_dims* dims, const void* q, const void* k_new,
+                                       const void* v_new, void* k_cache, void* v_cache,
+                                       void* desc, const int32_t* lens, int64_t len_bound,
+                                       double r, int32_t n_min, float softmax_scale, void* out,
+                                       float* lse, int32_t* sel, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* resa_decode_dense with row b at length lens[b]. */
+RESA_API int resa_decode_dense_varlen(const resa_dims* dims, const void* q, const void* k_new,
+                                      const void* v_new, void* k_cache, void* v_cache,
+                                      void* desc, const int32_t* lens, int64_t len_bound,
+                                      float softmax_scale, void* out, float* lse,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* resa_rectify with row b at length lens[b]: slots [lens[b]-f, lens[b]) are
+ * rewritten and out_f[b][i] sees keys 0 .. lens[b]-f+i. A row with
+ * lens[b] < f is left untouched (cache, descriptors and out_f), after
+ * clamping as above. Requires 1 <= f <= len_bound and f <= 256. */
+RESA_API int resa_rectify_varlen(const resa_dims* dims, const void* q_f, const void* k_f,
+                                 const void* v_f, void* k_cache, void* v_cache, void* desc,
+                                 const int32_t* lens, int64_t len_bound, int32_t f,
+                                 float softmax_scale, void* out_f, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * workspace control block. Returns RESA_OK, RESA_ERR_TIMEOUT,

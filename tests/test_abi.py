@@ -134,3 +134,50 @@ def test_status_strings(resa):
     for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert resa.status_string(code) != "unknown status"
     assert resa.status_string(-99) == "unknown status"
+
+
+def test_varlen_calls_reject_invalid_arguments(resa):
+    """The *_varlen calls need a 4-byte aligned lens array and apply the
+    fixed-length checks to len_bound; nothing is launched when they fail."""
+    E = resa
+    d = _dims(resa)
+    lib = resa._lib
+    dr = ctypes.byref(d)
+
+    def dec(lens=FAKE, bound=100, ws_bytes=1 << 30, r=0.1):
+        return lib.resa_decode_sparse_varlen(dr, FAKE, None, None, FAKE, FAKE, FAKE, lens, bound,
+                                             r, 4, 1.0, FAKE, None, None, FAKE, ws_bytes, None)
+    assert dec(lens=None) == E.RESA_ERR_INVALID_ARG
+    assert dec(lens=FAKE + 2) == E.RESA_ERR_INVALID_ARG
+    assert dec(bound=0) == E.RESA_ERR_INVALID_ARG
+    assert dec(bound=4097) == E.RESA_ERR_CAPACITY
+    assert dec(ws_bytes=512) == E.RESA_ERR_WORKSPACE
+    assert dec(r=0.0) == E.RESA_ERR_INVALID_ARG
+
+    def dense(lens=FAKE, bound=100):
+        return lib.resa_decode_dense_varlen(dr, FAKE, None, None, FAKE, FAKE, None, lens, bound,
+                                            1.0, FAKE, None, FAKE, 1 << 30, None)
+    assert dense(lens=None) == E.RESA_ERR_INVALID_ARG
+    assert dense(bound=4097) == E.RESA_ERR_CAPACITY
+
+    def rect(lens=FAKE, bound=100, f=32):
+        return lib.resa_rectify_varlen(dr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, lens, bound, f,
+                                       1.0, FAKE, FAKE, 1 << 30, None)
+    assert rect(lens=None) == E.RESA_ERR_INVALID_ARG
+    assert rect(f=101) == E.RESA_ERR_INVALID_ARG
+    assert rect(f=0) == E.RESA_ERR_INVALID_ARG
+    assert rect(bound=4097) == E.RESA_ERR_CAPACITY
+
+    assert lib.resa_build_desc_varlen(dr, FAKE, None, 100, FAKE, None) == E.RESA_ERR_INVALID_ARG
+    assert lib.resa_build_desc_varlen(dr, FAKE, FAKE, 4097, FAKE, None) == E.RESA_ERR_CAPACITY
+    assert lib.resa_build_desc_varlen(dr, FAKE, FAKE, 0, FAKE, None) == E.RESA_ERR_INVALID_ARG
+
+
+def test_workspace_covers_every_smaller_window(resa):
+    """A workspace sized for window f serves every window f' <= f (a smaller
+    window may take more splits per row)."""
+    for kw in (dict(batch=5), dict(batch=1), dict(batch=3, n_q_heads=12, n_kv_heads=4)):
+        d = _dims(resa, **kw)
+        big = resa.workspace_bytes(d, 4000, 64)
+        for f in range(1, 65):
+            assert resa.workspace_bytes(d, 4000, f) <= big, (kw, f)

@@ -1,0 +1,301 @@
+"""Ragged batches: every *_varlen call against one oracle state per row.
+
+Batch rows are independent sequences, so the oracle runs each row on its own
+(a batch of one at that row's length) and the GPU result of row b must match
+it exactly as a fixed-length call at that length would.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from pair import check_selection, close, tdt, to_dev
+from workload import Spec, decode_inputs, make_cache, ragged, rectify_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def resa():
+    import __graft_entry__
+    __graft_entry__.build()
+    import block_sparse_attention_quest_b200 as m
+    return m
+
+
+class VarPair:
+    """GPU tensors for a ragged batch + one oracle State per row."""
+
+    def __init__(self, resa, spec: Spec, lens0, r=None, n_min=None, bound=None):
+        self.resa, self.spec = resa, spec
+        self.r = spec.r if r is None else r
+        self.n_min = spec.n_min if n_min is None else n_min
+        self.fixed_bound = bound          # None: the longest row
+        K, V = ragged(*make_cache(spec), lens0)
+        self.states = [orc.State(K[b:b + 1], V[b:b + 1], int(n), spec.group)
+                       for b, n in enumerate(lens0)]
+        self.lens = np.asarray(lens0, dtype=np.int64)
+        self.k, self.v = to_dev(K, spec.dtype), to_dev(V, spec.dtype)
+        self.desc = torch.zeros(spec.batch, spec.n_kv_heads, spec.max_blocks, 2, spec.head_dim,
+                                dtype=tdt(spec.dtype), device="cuda")
+        resa.build_desc_varlen(self.k, self.lens_t(), self.bound(), self.desc, spec.n_q_heads)
+        self.dims = resa.dims_for(self.k, spec.n_q_heads)
+        self.ws = resa.alloc_workspace(self.dims, spec.max_len, max(spec.f, 64))
+        self.rect_calls = 0
+
+    def bound(self) -> int:
+        return int(self.lens.max()) if self.fixed_bound is None else self.fixed_bound
+
+    def lens_t(self):
+        return torch.tensor(self.lens, dtype=torch.int32, device="cuda")
+
+    def desc_matches(self):
+        d = self.desc.float().cpu().numpy()
+        for b, st in enumerate(self.states):
+            M = orc.num_blocks(st.length)
+            assert np.array_equal(d[b, :, :M, 0], st.lo[0, :, :M]), f"row {b} min"
+            assert np.array_equal(d[b, :, :M, 1], st.hi[0, :, :M]), f"row {b} max"
+            assert not d[b, :, M:].any(), f"row {b}: blocks past its length were written"
+
+    def decode(self, step: int, dense: bool = False, scale: float = 1.0):
+        spec, resa = self.spec, self.resa
+        q, kn, vn = decode_inputs(spec, step)
+        self.lens += 1
+        B = spec.batch
+        out = torch.empty(B, spec.n_q_heads, spec.head_dim, dtype=tdt(spec.dtype), device="cuda")
+        lse = torch.empty(B, spec.n_q_heads, dtype=torch.float32, device="cuda")
+        args = (to_dev(q, spec.dtype), to_dev(kn, spec.dtype), to_dev(vn, spec.dtype), self.k,
+                self.v, self.desc, self.lens_t(), self.bound())
+        sel = None
+        if dense:
+            resa.decode_dense_varlen(*args, scale, out, self.ws, lse=lse)
+        else:
+            n_cap = resa.num_selected(self.bound(), self.r, self.n_min)
+            sel = torch.full((B, spec.n_kv_heads, n_cap), -7, dtype=torch.int32, device="cuda")
+            resa.decode_sparse_varlen(*args, self.r, self.n_min, scale, out, self.ws, lse=lse,
+                                      sel=sel)
+        assert resa.workspace_status(self.ws) == resa.RESA_OK
+        out = out.float().cpu().numpy()
+        lse = lse.cpu().numpy()
+        gsel = None if sel is None else sel.cpu().numpy()
+        for b, st in enumerate(self.states):
+            qb, kb, vb = q[b:b + 1], kn[b:b + 1], vn[b:b + 1]
+            if dense:
+                st.append(kb, vb)
+                O, L = st.dense(qb, scale)
+            else:
+                res = st.decode(qb, kb, vb, self.r, self.n_min, scale)
+                n_b = res["n"]
+                assert (gsel[b, :, n_b:] == -1).all(), f"row {b}: list tail must be -1"
+                exact = True
+                for g in range(spec.n_kv_heads):
+                    exact &= check_selection(gsel[b, g, :n_b], res["scores"][0, g], n_b)
+                O, L = res["out"], res["lse"]
+                if not exact:
+                    O, L = st.attend_with(qb, gsel[b:b + 1, :, :n_b], scale)
+            close(out[b], O[0], spec.dtype, f"row {b} (len {st.length}) step {step} out")
+            close(lse[b], L[0], "f32" if spec.dtype == "f32" else "bf16",
+                  f"row {b} step {step} lse")
+        return gsel
+
+    def rectify(self, f: int, scale: float = 1.0):
+        spec, resa = self.spec, self.resa
+        q_f, k_f, v_f = rectify_inputs(spec, self.rect_calls, self.bound(), f)
+        self.rect_calls += 1
+        sentinel = 3.0
+        out = torch.full((spec.batch, f, spec.n_q_heads, spec.head_dim), sentinel,
+                         dtype=tdt(spec.dtype), device="cuda")
+        before = (self.k.clone(), self.v.clone(), self.desc.clone())
+        resa.rectify_varlen(to_dev(q_f, spec.dtype), to_dev(k_f, spec.dtype),
+                            to_dev(v_f, spec.dtype), self.k, self.v, self.desc, self.lens_t(),
+                            self.bound(), f, scale, out, self.ws)
+        assert resa.workspace_status(self.ws) == resa.RESA_OK
+        got = out.float().cpu().numpy()
+        for b, st in enumerate(self.states):
+            if st.length < f:   # shorter than the window: left untouched
+                assert (got[b] == sentinel).all(), f"row {b}: output written"
+                for new, old in zip((self.k, self.v, self.desc), before):
+                    assert torch.equal(new[b], old[b]), f"row {b}: cache touched"
+                continue
+            ref = st.rectify(q_f[b:b + 1], k_f[b:b + 1], v_f[b:b + 1], f, scale)
+            close(got[b], ref[0], spec.dtype, f"row {b} (len {st.length}) rectify f={f}")
+
+
+def test_varlen_bf16_decode_and_rectify(resa):
+    """Rows of 5000, 1234, 17, 3001 and 4096 tokens (a partial single-block
+    row, a block-aligned row), 32 sparse steps, a rectify, 6 more steps."""
+    spec = Spec(batch=5, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=5000, steps=40)
+    p = VarPair(resa, spec, [5000, 1234, 17, 3001, 4096])
+    p.desc_matches()
+    for step in range(32):
+        p.decode(step)
+    p.desc_matches()
+    p.rectify(32)
+    p.desc_matches()
+    for step in range(32, 38):
+        p.decode(step)
+    p.desc_matches()
+
+
+def test_varlen_f32_dense_rows_and_short_rectify(resa):
+    """fp32 (CUDA-core kernels), rows down to 5 tokens; a rectify window
+    longer than one row leaves that row alone; then dense decode."""
+    spec = Spec(batch=3, n_q_heads=8, n_kv_heads=2, head_dim=64, len0=1000, steps=40,
+                dtype="f32", r=0.1, n_min=4, rect_block_mean=False)
+    p = VarPair(resa, spec, [300, 5, 1000])
+    p.desc_matches()
+    for step in range(16):
+        p.decode(step)
+    p.rectify(16)            # every row has >= 16 tokens now
+    p.rectify(32)            # the 21-token row is shorter than the window
+    p.desc_matches()
+    for step in range(16, 20):
+        p.decode(step, dense=True)
+    p.desc_matches()
+
+
+def test_varlen_group3_rectify_fallback_and_fixed_bound(resa):
+    """bf16 with G = 3 (rectify on the split-KV kernel), a bound above every
+    row (the capacity), so every row is shorter than the grid's bound."""
+    spec = Spec(batch=3, n_q_heads=12, n_kv_heads=4, head_dim=64, len0=2100, steps=40, r=0.2,
+                n_min=8)
+    p = VarPair(resa, spec, [700, 2100, 64], bound=spec.max_len)
+    for step in range(32):
+        p.decode(step)
+    p.rectify(32)
+    p.desc_matches()
+    p.decode(32)
+
+
+def test_varlen_equal_lengths_match_fixed_length_call_bitwise(resa):
+    """With every row at the same length the ragged call is the fixed-length
+    call: same kernels, same splits, identical bits."""
+    spec = Spec(batch=2, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=6000, steps=2)
+    K, V = make_cache(spec)
+    ka, va = to_dev(K, "bf16"), to_dev(V, "bf16")
+    kb, vb = ka.clone(), va.clone()
+    da = torch.zeros(2, 8, spec.max_blocks, 2, 128, dtype=torch.bfloat16, device="cuda")
+    db = torch.zeros_like(da)
+    lens = torch.full((2,), 6000, dtype=torch.int32, device="cuda")
+    resa.build_desc(ka, 6000, da, 32)
+    resa.build_desc_varlen(kb, lens, 6000, db, 32)
+    assert torch.equal(da, db)
+    dims = resa.dims_for(ka, 32)
+    wa, wb = resa.alloc_workspace(dims, spec.max_len, 32), resa.alloc_workspace(dims, spec.max_len, 32)
+    q, kn, vn = (to_dev(x, "bf16") for x in decode_inputs(spec, 0))
+    n = resa.num_selected(6001, spec.r, spec.n_min)
+    outs = []
+    for fixed in (True, False):
+        out = torch.empty(2, 32, 128, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(2, 32, dtype=torch.float32, device="cuda")
+        sel = torch.empty(2, 8, n, dtype=torch.int32, device="cuda")
+        if fixed:
+            resa.decode_sparse(q, kn, vn, ka, va, da, 6001, spec.r, spec.n_min, 1.0, out, wa,
+                               lse=lse, sel=sel)
+        else:
+            resa.decode_sparse_varlen(q, kn, vn, kb, vb, db, lens + 1, 6001, spec.r, spec.n_min,
+                                      1.0, out, wb, lse=lse, sel=sel)
+        outs.append((out, lse, sel))
+    for x, y in zip(*outs):
+        assert torch.equal(x, y)
+    assert torch.equal(ka, kb) and torch.equal(va, vb) and torch.equal(da, db)
+    q_f, k_f, v_f = (to_dev(x, "bf16") for x in rectify_inputs(spec, 0, 6001, 32))
+    ra = torch.empty(2, 32, 32, 128, dtype=torch.bfloat16, device="cuda")
+    rb = torch.empty_like(ra)
+    resa.rectify(q_f, k_f, v_f, ka, va, da, 6001, 32, 1.0, ra, wa)
+    resa.rectify_varlen(q_f, k_f, v_f, kb, vb, db, lens + 1, 6001, 32, 1.0, rb, wb)
+    assert torch.equal(ra, rb)
+    assert torch.equal(ka, kb) and torch.equal(va, vb) and torch.equal(da, db)
+
+
+def test_varlen_select_beyond_register_path(resa):
+    """A bound above 16384 blocks sends selection to the shared-memory radix
+    kernel; a 300000-token row and a 100003-token row share one call."""
+    spec = Spec(batch=2, n_q_heads=8, n_kv_heads=1, head_dim=64, len0=300000, steps=2, r=0.05,
+                n_min=16)
+    p = VarPair(resa, spec, [300000, 100003])
+    p.decode(0)
+    p.decode(1)
+    p.desc_matches()
+
+
+def test_varlen_graph_replay_with_changing_lengths(resa):
+    """lens is read on the device only: one captured decode replays correctly
+    while the row lengths (and so M, n and the appended slot) change."""
+    spec = Spec(batch=3, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=3000, steps=12)
+    p = VarPair(resa, spec, [3000, 811, 2040], bound=spec.max_len)
+    B, dt = spec.batch, tdt(spec.dtype)
+    q_s = torch.zeros(B, 32, 128, dtype=dt, device="cuda")
+    kn_s = torch.zeros(B, 8, 128, dtype=dt, device="cuda")
+    vn_s = torch.zeros_like(kn_s)
+    lens_s = p.lens_t()
+    n_cap = resa.num_selected(spec.max_len, p.r, p.n_min)
+    out = torch.empty(B, 32, 128, dtype=dt, device="cuda")
+    lse = torch.empty(B, 32, dtype=torch.float32, device="cuda")
+    sel = torch.empty(B, 8, n_cap, dtype=torch.int32, device="cuda")
+
+    def call():
+        resa.decode_sparse_varlen(q_s, kn_s, vn_s, p.k, p.v, p.desc, lens_s, spec.max_len, p.r,
+                                  p.n_min, 1.0, out, p.ws, lse=lse, sel=sel)
+
+    # one eager call on copies first, so that every one-time host setup
+    # (kernel attributes, occupancy queries) happens outside the capture
+    kw, vw, dw = p.k.clone(), p.v.clone(), p.desc.clone()
+    ws_w = resa.alloc_workspace(p.dims, spec.max_len, 64)
+    resa.decode_sparse_varlen(q_s, kn_s, vn_s, kw, vw, dw, lens_s + 1, spec.max_len, p.r,
+                              p.n_min, 1.0, out, ws_w, lse=lse, sel=sel)
+    assert resa.workspace_status(ws_w) == resa.RESA_OK
+    # the captured work itself does not run during capture
+    k0, v0, d0 = p.k.clone(), p.v.clone(), p.desc.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            call()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    assert torch.equal(p.k, k0) and torch.equal(p.v, v0) and torch.equal(p.desc, d0)
+    for step in range(8):
+        q, kn, vn = decode_inputs(spec, step)
+        p.lens += 1
+        q_s.copy_(to_dev(q, spec.dtype))
+        kn_s.copy_(to_dev(kn, spec.dtype))
+        vn_s.copy_(to_dev(vn, spec.dtype))
+        lens_s.copy_(p.lens_t())
+        g.replay()
+        torch.cuda.synchronize()
+        assert resa.workspace_status(p.ws) == resa.RESA_OK
+        got, gl, gsel = out.float().cpu().numpy(), lse.cpu().numpy(), sel.cpu().numpy()
+        for b, st in enumerate(p.states):
+            res = st.decode(q[b:b + 1], kn[b:b + 1], vn[b:b + 1], p.r, p.n_min, 1.0)
+            n_b = res["n"]
+            assert (gsel[b, :, n_b:] == -1).all()
+            exact = all([check_selection(gsel[b, gg, :n_b], res["scores"][0, gg], n_b)
+                         for gg in range(8)])
+            O, L = res["out"], res["lse"]
+            if not exact:
+                O, L = st.attend_with(q[b:b + 1], gsel[b:b + 1, :, :n_b], 1.0)
+            close(got[b], O[0], spec.dtype, f"replay {step} row {b}")
+            close(gl[b], L[0], "bf16", f"replay {step} row {b} lse")
+    del g
+    p.desc_matches()
+
+
+def test_varlen_out_of_range_lengths_are_clamped_and_flagged(resa):
+    """Entries outside [1, len_bound] are clamped on the device (every access
+    stays inside the row) and reported through the workspace flag."""
+    spec = Spec(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=64, len0=512, steps=2)
+    p = VarPair(resa, spec, [512, 100])
+    dt = tdt(spec.dtype)
+    q, kn, vn = (to_dev(x, spec.dtype) for x in decode_inputs(spec, 0))
+    out = torch.empty(2, 8, 64, dtype=dt, device="cuda")
+    bad = torch.tensor([600, 0], dtype=torch.int32, device="cuda")   # above the bound, below 1
+    resa.decode_sparse_varlen(q, kn, vn, p.k, p.v, p.desc, bad, 513, p.r, p.n_min, 1.0, out, p.ws)
+    assert resa.workspace_status(p.ws) == resa.RESA_ERR_BAD_INDEX
+    assert torch.isfinite(out.float()).all()
+    assert resa.workspace_status(p.ws) == resa.RESA_OK     # the flag was cleared
+    q_f, k_f, v_f = (to_dev(x, spec.dtype) for x in rectify_inputs(spec, 0, 513, 16))
+    out_f = torch.empty(2, 16, 8, 64, dtype=dt, device="cuda")
+    resa.rectify_varlen(q_f, k_f, v_f, p.k, p.v, p.desc, bad, 513, 16, 1.0, out_f, p.ws)
+    assert resa.workspace_status(p.ws) == resa.RESA_ERR_BAD_INDEX

@@ -40,6 +40,7 @@ _S_CACHE_K, _S_CACHE_V, _S_MEAN_K, _S_MEAN_V = 1, 2, 3, 4
 _S_Q, _S_KNEW, _S_VNEW = 5, 6, 7
 _S_RQ, _S_RK, _S_RV = 8, 9, 10
 _S_NEEDLE = 11
+_S_LENS = 12
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -158,6 +159,26 @@ def make_cache(spec: Spec):
                 for j in pos[b, h]:
                     K[b, h, j * BLOCK:(j + 1) * BLOCK] += spec.needle_shift * qd[b, h]
     return round_to(K, spec.dtype), round_to(V, spec.dtype)
+
+
+def length_mix(spec: Spec, min_len: int, salt: int = 0) -> np.ndarray:
+    """Per-row prompt lengths for a ragged batch: int32 [B] drawn uniformly
+    from [min_len, spec.len0]; the longest row is set to spec.len0 so that
+    spec.len0 stays the bound."""
+    g = _rng(spec.seed, _S_LENS, salt)
+    lens = g.integers(min_len, spec.len0 + 1, size=spec.batch).astype(np.int32)
+    lens[int(g.integers(0, spec.batch))] = spec.len0
+    return lens
+
+
+def ragged(K: np.ndarray, V: np.ndarray, lens0) -> tuple[np.ndarray, np.ndarray]:
+    """Copies of K, V [B, Hkv, L, d] with row b's slots at or past lens0[b]
+    cleared, as a cache filled to those lengths would be."""
+    K, V = K.copy(), V.copy()
+    for b, n in enumerate(lens0):
+        K[b, :, int(n):] = 0.0
+        V[b, :, int(n):] = 0.0
+    return K, V
 
 
 def decode_inputs(spec: Spec, step: int):
