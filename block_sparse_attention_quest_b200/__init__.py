@@ -90,7 +90,7 @@ _lib.resa_decode_dense_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, 
                                           ctypes.c_int64, ctypes.c_float, _P, _P, _P,
                                           ctypes.c_size_t, _P]
 _lib.resa_rectify_varlen.restype = ctypes.c_int
-_lib.resa_rectify_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P,
+_lib.resa_rectify_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P,
                                      ctypes.c_size_t, _P]
 _lib.resa_workspace_status.restype = ctypes.c_int
@@ -267,9 +267,11 @@ def decode_dense_varlen(q, k_new, v_new, k_cache, v_cache, desc, lens, len_bound
 
 
 def rectify_varlen(q_f, k_f, v_f, k_cache, v_cache, desc, lens, len_bound: int, f: int,
-                   softmax_scale: float, out_f, workspace, stream=None) -> None:
+                   softmax_scale: float, out_f, workspace, windows=None, stream=None) -> None:
+    """windows: optional int32 CUDA tensor [batch] of per-row windows in [0, f]
+    (0 = row not rectified); None = every row uses f."""
     dims = dims_for(k_cache, q_f.shape[2])
     _check(_lib.resa_rectify_varlen(
         ctypes.byref(dims), _ptr(q_f), _ptr(k_f), _ptr(v_f), _ptr(k_cache), _ptr(v_cache),
-        _ptr(desc), _lens(lens), int(len_bound), int(f), float(softmax_scale), _ptr(out_f),
+        _ptr(desc), _lens(lens), None if windows is None else _lens(windows), int(len_bound), int(f), float(softmax_scale), _ptr(out_f),
         _ptr(workspace), workspace.numel(), _stream(stream)), "resa_rectify_varlen")

@@ -196,7 +196,8 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? RESA_OK : RESA_ERR_CU
 int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int32_t* sel, int n_sel,
                   float scale, const void* k, const void* v, void* out, float* lse, uint8_t* ws,
                   const WsLayout& w, int num_sms, cudaStream_t st, bool pdl = false,
-                  const int32_t* lens = nullptr, double r = 0.0, int n_min = 0) {
+                  const int32_t* lens = nullptr, double r = 0.0, int n_min = 0,
+                  const int32_t* windows = nullptr) {
   const int64_t min_blocks = sel ? n_sel : blocks_of(len0);
   const int S = splits_for(s.B * s.H * R, min_blocks, num_sms, s);
   AttnArgs a{};
@@ -209,7 +210,7 @@ int run_attention(const Shape& s, const void* q, int R, int64_t len0, const int3
   a.ctrl = reinterpret_cast<Ctrl*>(ws);
   a.k = k; a.v = v;
   a.pdl = pdl;
-  a.lens = lens; a.r = r; a.n_min = n_min;
+  a.lens = lens; a.windows = windows; a.r = r; a.n_min = n_min;
   CUtensorMap tk, tv;
   if (s.bf16) {
     if (!make_cache_map(&tk, k, s) || !make_cache_map(&tv, v, s)) return RESA_ERR_CUDA;
@@ -462,7 +463,8 @@ int resa_decode_dense_varlen(const resa_dims* dims, const void* q, const void* k
 static int rectify_impl(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
                         void* k_cache, void* v_cache, void* desc, int64_t len, int32_t f,
                         float softmax_scale, void* out_f, void* workspace,
-                        size_t workspace_bytes, void* stream, const int32_t* lens) {
+                        size_t workspace_bytes, void* stream, const int32_t* lens,
+                        const int32_t* windows) {
   Shape s;
   int rc = check_dims(dims, &s);
   if (rc != RESA_OK) return rc;
@@ -478,7 +480,7 @@ static int rectify_impl(const resa_dims* dims, const void* q_f, const void* k_f,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, f);
   cudaError_t e = launch_rectify_write(s, k_f, v_f, k_cache, v_cache, desc, len, f, st, lens,
-                                       reinterpret_cast<Ctrl*>(ws));
+                                       windows, reinterpret_cast<Ctrl*>(ws));
   if (e != cudaSuccess) return RESA_ERR_CUDA;
   if (rectify_on_tensor_cores(s)) {
     RectArgs r{};
@@ -490,7 +492,7 @@ static int rectify_impl(const resa_dims* dims, const void* q_f, const void* k_f,
     if (S > kMaxSplits) S = kMaxSplits;
     if (S > n_tiles) S = n_tiles;
     r.S = static_cast<int>(S);
-    r.len = len; r.lens = lens; r.L_max = s.L_max; r.scale = softmax_scale; r.out = out_f;
+    r.len = len; r.lens = lens; r.windows = windows; r.L_max = s.L_max; r.scale = softmax_scale; r.out = out_f;
     r.part_o = reinterpret_cast<float*>(ws + w.part_o);
     r.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
     r.ctrl = reinterpret_cast<Ctrl*>(ws);
@@ -502,7 +504,7 @@ static int rectify_impl(const resa_dims* dims, const void* q_f, const void* k_f,
     return cuda_status(launch_rectify_tc(r, st));
   }
   return run_attention(s, q_f, f, len - f + 1, nullptr, 0, softmax_scale, k_cache, v_cache, out_f,
-                       nullptr, ws, w, num_sms, st, false, lens);
+                       nullptr, ws, w, num_sms, st, false, lens, 0.0, 0, windows);
 }
 
 int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const void* v_f,
@@ -510,16 +512,17 @@ int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_f, const 
                  float softmax_scale, void* out_f, void* workspace, size_t workspace_bytes,
                  void* stream) {
   return rectify_impl(dims, q_f, k_f, v_f, k_cache, v_cache, desc, len, f, softmax_scale, out_f,
-                      workspace, workspace_bytes, stream, nullptr);
+                      workspace, workspace_bytes, stream, nullptr, nullptr);
 }
 
 int resa_rectify_varlen(const resa_dims* dims, const void* q_f, const void* k_f,
                         const void* v_f, void* k_cache, void* v_cache, void* desc,
-                        const int32_t* lens, int64_t len_bound, int32_t f, float softmax_scale,
-                        void* out_f, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!lens_ok(lens)) return RESA_ERR_INVALID_ARG;
+                        const int32_t* lens, const int32_t* windows, int64_t len_bound,
+                        int32_t f, float softmax_scale, void* out_f, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!lens_ok(lens) || (windows != nullptr && !lens_ok(windows))) return RESA_ERR_INVALID_ARG;
   return rectify_impl(dims, q_f, k_f, v_f, k_cache, v_cache, desc, len_bound, f, softmax_scale,
-                      out_f, workspace, workspace_bytes, stream, lens);
+                      out_f, workspace, workspace_bytes, stream, lens, windows);
 }
 
 int resa_workspace_status(void* workspace, void* stream) {

@@ -38,21 +38,29 @@ struct AttnK {
   int64_t len0;
   int64_t L_max;
   const int32_t* lens;   // optional per-row lengths [B] (see AttnArgs)
+  const int32_t* windows;  // optional per-row query counts [B] (see AttnArgs)
   double r;
   int n_min;
   int R, Hq, H, G, n_sel, S;
   float scale_log2;
 };
 
-// Tokens visible to query row r of batch row b (the last row sees the whole
-// row); <= 0 when the batch row is shorter than the query rows.
-__device__ __forceinline__ int64_t query_len(const AttnK& a, int b, int r) {
-  if (a.lens == nullptr) return a.len0 + r;
-  return row_len(a.lens, a.len0 + a.R - 1, b) - (a.R - 1) + r;
+// Query rows of batch row b in use (all R unless per-row windows are given).
+__device__ __forceinline__ int query_rows(const AttnK& a, int b) {
+  return row_window(a.windows, a.R, b);
 }
-// a batch row shorter than its query rows is skipped (variable lengths only)
-__device__ __forceinline__ bool row_skipped(const AttnK& a, int b) {
-  return a.lens != nullptr && row_len(a.lens, a.len0 + a.R - 1, b) < a.R;
+// Tokens visible to query row r of batch row b: the row's last query row
+// sees the whole row.
+__device__ __forceinline__ int64_t query_len(const AttnK& a, int b, int r) {
+  if (a.lens == nullptr && a.windows == nullptr) return a.len0 + r;
+  return row_len(a.lens, a.len0 + a.R - 1, b) - query_rows(a, b) + 1 + r;
+}
+// query rows past the batch row's count, and batch rows shorter than their
+// count (or with count 0), are skipped (variable lengths and windows only)
+__device__ __forceinline__ bool row_skipped(const AttnK& a, int b, int r) {
+  if (a.lens == nullptr && a.windows == nullptr) return false;
+  const int w = query_rows(a, b);
+  return r >= w || row_len(a.lens, a.len0 + a.R - 1, b) < w;
 }
 
 constexpr int kIdCache = 1024;   // block ids of one CTA kept in shared memory
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
   const int b = br / a.R, r = br % a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (row_skipped(a, b)) return;
+  if (row_skipped(a, b, r)) return;
   const int64_t len_r = query_len(a, b, r);
   int i0, i1;
   split_range(a, s_idx, len_r, i0, i1);
@@ -446,7 +454,7 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
   const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
   const int b = br / a.R, r = br % a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (row_skipped(a, b)) return;
+  if (row_skipped(a, b, r)) return;
   const int64_t len_r = query_len(a, b, r);
   const float* qrow = static_cast<const float*>(a.q) + (static_cast<int64_t>(br) * a.Hq + g * a.G) * D;
   for (int i = threadIdx.x; i < a.G * D; i += NW * 32) sq[i] = qrow[i];
@@ -613,7 +621,7 @@ cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st) {
   k.counters = a.counters; k.out = a.out; k.lse = a.lse;
   k.k = a.k; k.v = a.v; k.len0 = a.len0; k.L_max = s.L_max; k.R = a.R; k.Hq = s.Hq; k.H = s.H;
   k.G = s.G; k.n_sel = a.n_sel; k.S = a.S;
-  k.lens = a.lens; k.r = a.r; k.n_min = a.n_min;
+  k.lens = a.lens; k.windows = a.windows; k.r = a.r; k.n_min = a.n_min;
   k.scale_log2 = a.scale * 1.4426950408889634f;
   if (s.bf16) return s.D == 128 ? attend_bf16_t<128>(s, k, a, st) : attend_bf16_t<64>(s, k, a, st);
   return s.D == 128 ? attend_f32_t<128>(s, k, a, st) : attend_f32_t<64>(s, k, a, st);

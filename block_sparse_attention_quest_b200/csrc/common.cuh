@@ -44,6 +44,17 @@ __device__ __forceinline__ int64_t row_len(const int32_t* lens, int64_t len, int
 __device__ __forceinline__ bool row_len_bad(const int32_t* lens, int64_t len, int b) {
   return lens != nullptr && (lens[b] < 1 || static_cast<int64_t>(lens[b]) > len);
 }
+// Rectify window of batch row b: windows[b] when given (clamped to [0, f]),
+// else f. A row with window 0, or shorter than its window, is not rectified.
+__device__ __forceinline__ int row_window(const int32_t* windows, int f, int b) {
+  if (windows == nullptr) return f;
+  const int w = windows[b];
+  return w < 0 ? 0 : (w > f ? f : w);
+}
+__device__ __forceinline__ bool row_window_bad(const int32_t* windows, int f, int b) {
+  return windows != nullptr && (windows[b] < 0 || windows[b] > f);
+}
+
 // Block budget of Eq. 5 on the device; the same double-precision formula as
 // resa_num_selected: n = min(M, max(n_min, ceil(M r - 1e-9))).
 __device__ __forceinline__ int num_selected_dev(int64_t len, double r, int n_min) {

@@ -102,14 +102,17 @@ template <typename T>
 __global__ void rectify_write_kernel(const T* __restrict__ k_f, const T* __restrict__ v_f,
                                      T* __restrict__ k, T* __restrict__ v, T* __restrict__ desc,
                                      int H, int D, int64_t L_max, int Mmax, int64_t len, int f,
-                                     const int32_t* lens, Ctrl* ctrl) {
+                                     const int32_t* lens, const int32_t* windows, Ctrl* ctrl) {
   const int c = threadIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * H + h;
-  if (blockIdx.x == 0 && h == 0 && c == 0 && row_len_bad(lens, len, b)) raise_error(ctrl, kErrBadIndex);
+  if (blockIdx.x == 0 && h == 0 && c == 0 &&
+      (row_len_bad(lens, len, b) || row_window_bad(windows, f, b)))
+    raise_error(ctrl, kErrBadIndex);
   len = row_len(lens, len, b);
-  if (len < f) return;                     // a row shorter than the window is left alone
-  const int64_t t_first = len - f;
+  const int w = row_window(windows, f, b);  // this row's window (rows w .. f-1 of k_f unused)
+  if (w == 0 || len < w) return;            // not rectified: left alone
+  const int64_t t_first = len - w;
   const int64_t j = t_first / kBlock + blockIdx.x;
   if (j * kBlock >= len) return;           // this row touches fewer blocks
   const int64_t t0 = j * kBlock;
@@ -177,22 +180,23 @@ cudaError_t launch_append(const Shape& s, const void* k_new, const void* v_new, 
 
 cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_f, void* k, void* v,
                                  void* desc, int64_t len, int f, cudaStream_t st,
-                                 const int32_t* lens, Ctrl* ctrl) {
+                                 const int32_t* lens, const int32_t* windows, Ctrl* ctrl) {
   // blocks touched by f slots: at most f/16 + 2 (the bound covers every row)
   const int64_t j0 = (len - f) / kBlock;
   const int64_t M = (len + kBlock - 1) / kBlock;
-  const int64_t touched = lens ? f / kBlock + 2 : M - j0;
+  const int64_t touched = (lens || windows) ? f / kBlock + 2 : M - j0;
   dim3 grid(static_cast<unsigned>(touched), s.H, s.B);
   if (s.bf16) {
     using T = __nv_bfloat16;
     rectify_write_kernel<T><<<grid, s.D, 0, st>>>(
         static_cast<const T*>(k_f), static_cast<const T*>(v_f), static_cast<T*>(k),
-        static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f, lens, ctrl);
+        static_cast<T*>(v), static_cast<T*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f, lens,
+        windows, ctrl);
   } else {
     rectify_write_kernel<float><<<grid, s.D, 0, st>>>(
         static_cast<const float*>(k_f), static_cast<const float*>(v_f), static_cast<float*>(k),
         static_cast<float*>(v), static_cast<float*>(desc), s.H, s.D, s.L_max, s.Mmax, len, f, lens,
-        ctrl);
+        windows, ctrl);
   }
   return cudaGetLastError();
 }

@@ -25,7 +25,8 @@ cudaError_t launch_append(const Shape& s, const void* k_new, const void* v_new, 
                           void* desc, int64_t len, cudaStream_t st, const int32_t* lens = nullptr);
 cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_f, void* k, void* v,
                                  void* desc, int64_t len, int f, cudaStream_t st,
-                                 const int32_t* lens = nullptr, Ctrl* ctrl = nullptr);
+                                 const int32_t* lens = nullptr, const int32_t* windows = nullptr,
+                                 Ctrl* ctrl = nullptr);
 
 // scoring + selection ----------------------------------------------------------
 // scores: [B][H][M] float; the CTA that owns the last chunk also performs the
@@ -60,10 +61,14 @@ struct AttnArgs {
   const void* v;
   bool pdl;               // launched as a programmatic dependent of the select kernel
   // optional per-row lengths [B]: row b's last query row sees lens[b] tokens
-  // (len0 + R - 1 is then their bound); a batch row shorter than R is
-  // skipped; selected rows hold Eq. 5's n for their own length (r, n_min),
-  // n_sel being the list stride
+  // (len0 + R - 1 is then their bound); selected rows hold Eq. 5's n for
+  // their own length (r, n_min), n_sel being the list stride
   const int32_t* lens;
+  // optional per-row query counts [B] (rectify windows, clamped to [0, R]):
+  // row b uses query rows 0 .. w-1 at positions lens[b] - w .. lens[b] - 1;
+  // without it every row uses all R. A batch row shorter than its count
+  // (or with count 0) is skipped.
+  const int32_t* windows;
   double r;
   int n_min;
 };
@@ -100,7 +105,9 @@ int fused_max_share();
 struct RectArgs {
   int B, H, Hq, G, D, f, S, mtiles;
   int64_t len, L_max;     // len: the cache length (with lens: the bound on the rows')
-  const int32_t* lens;    // optional per-row lengths [B]; rows shorter than f are skipped
+  const int32_t* lens;    // optional per-row lengths [B]
+  const int32_t* windows; // optional per-row windows [B] in [0, f]; rows with window 0 or
+                          // shorter than their window are skipped
   float scale;
   void* out;              // [B][f][Hq][D] bf16
   float* part_o;          // [B*f*Hq][S][D]

@@ -40,6 +40,7 @@ struct RectK {
   int64_t len;
   int64_t L_max;
   const int32_t* lens;   // optional per-row lengths [B] (len: their bound)
+  const int32_t* windows;  // optional per-row windows [B] in [0, f]
   int H, Hq, G, f, S, mtiles;
   float scale_log2;
 };
@@ -88,7 +89,9 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   const int b = blockIdx.z / a.mtiles, mt = blockIdx.z % a.mtiles;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t len = row_len(a.lens, a.len, b);
-  if (len < a.f) return;                   // a row shorter than the window is skipped
+  const int win = row_window(a.windows, a.f, b);   // query rows in use: 0 .. win-1
+  if (win == 0 || len < win) return;       // not rectified: skipped
+  if (mt * 128 >= win * a.G) return;       // this m-tile holds no row in use
   const int n_tiles = static_cast<int>((len + 127) / 128);
   const int t0 = static_cast<int>(static_cast<int64_t>(s_idx) * n_tiles / a.S);
   const int t1 = static_cast<int>(static_cast<int64_t>(s_idx + 1) * n_tiles / a.S);
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
     const int row = threadIdx.x & 127;                     // TMEM lane / tile row
     const int rg = mt * 128 + row;
     const int qi = rg / a.G, hh = rg % a.G;
-    const int64_t qpos = len - a.f + qi;                   // causal limit of this row
+    const int64_t qpos = len - win + qi;                   // causal limit of this row
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;                      // reference max (log2 units), sum
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       const int64_t key0 = static_cast<int64_t>(t0 + t) * 128;
       // keys above the smallest causal limit of the tile (or past the end of
       // the cache) exist only in the last tiles
-      const bool masked = key0 + 127 > len - a.f;
+      const bool masked = key0 + 127 > len - win;
       const int lim = masked ? static_cast<int>(qpos - key0 < 127 ? qpos - key0 : 127) : 127;
       // pass 1: row maximum of the raw scores
       float mx = -INFINITY;
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
       const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
       const float lt = a0 * l0 + a1 * l1;
-      const bool valid = qi < a.f;
+      const bool valid = qi < win;
       const int64_t orow = (static_cast<int64_t>(b) * a.f + qi) * a.Hq + g * a.G + hh;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -384,12 +387,18 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const float* __restrict
                                                          __nv_bfloat16* __restrict__ out,
                                                          int64_t rows, int S,
                                                          const int32_t* lens, int64_t len,
-                                                         int64_t rows_per_b, int f) {
+                                                         const int32_t* windows,
+                                                         int64_t rows_per_b, int f, int Hq) {
   constexpr int CPL = D / 32;
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
-  if (lens != nullptr && row_len(lens, len, static_cast<int>(row / rows_per_b)) < f) return;
+  if (lens != nullptr || windows != nullptr) {
+    const int b = static_cast<int>(row / rows_per_b);
+    const int w = row_window(windows, f, b);
+    const int qi = static_cast<int>((row % rows_per_b) / Hq);
+    if (qi >= w || row_len(lens, len, b) < w) return;   // row not rectified
+  }
   const float* ml = part_ml + row * S * 2;
   float mstar = -INFINITY;
   for (int s = lane; s < S; s += 32) mstar = fmaxf(mstar, ml[2 * s]);
@@ -448,7 +457,7 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   RectK k{};
   k.out = r.out; k.part_o = r.part_o; k.part_ml = r.part_ml; k.ctrl = r.ctrl;
   k.len = r.len; k.L_max = r.L_max; k.H = r.H; k.Hq = r.Hq; k.G = r.G; k.f = r.f; k.S = r.S;
-  k.lens = r.lens;
+  k.lens = r.lens; k.windows = r.windows;
   k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
   dim3 grid(r.S, r.H, r.B * r.mtiles);
   rectify_tc_kernel<D><<<grid, 288, C::kSmem, st>>>(*r.tm_q, *r.tm_k, *r.tm_v, k);
@@ -457,7 +466,7 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(r.B) * r.f * r.Hq;
   merge_rows_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(
       r.part_o, r.part_ml, static_cast<__nv_bfloat16*>(r.out), rows, r.S, r.lens, r.len,
-      static_cast<int64_t>(r.f) * r.Hq, r.f);
+      r.windows, static_cast<int64_t>(r.f) * r.Hq, r.f, r.Hq);
   return cudaGetLastError();
 }
 

@@ -239,14 +239,21 @@ RESA_API int resa_decode_dense_varlen(const resa_dims* dims, const void* q, cons
                                       float softmax_scale, void* out, float* lse,
                                       void* workspace, size_t workspace_bytes, void* stream);
 
-/* resa_rectify with row b at length lens[b]: slots [lens[b]-f, lens[b]) are
- * rewritten and out_f[b][i] sees keys 0 .. lens[b]-f+i. A row with
- * lens[b] < f is left untouched (cache, descriptors and out_f), after
- * clamping as above. Requires 1 <= f <= len_bound and f <= 256. */
+/* resa_rectify with row b at length lens[b] and its own window w_b, so rows
+ * can sit at different rectification phases: w_b = windows[b] (device int32
+ * [batch], 4-byte aligned), or f for every row when windows is NULL. Row b
+ * uses the first w_b rows of its q_f/k_f/v_f block ([batch][f][..] as in
+ * resa_rectify): slots [lens[b]-w_b, lens[b]) are rewritten, the blocks they
+ * touch refreshed, and out_f[b][i] (i < w_b) is the causal dense attention of
+ * q_f[b][i] at position lens[b]-w_b+i. Rows i >= w_b of out_f are not
+ * written. A row with w_b = 0, or with lens[b] < w_b, is left untouched
+ * (cache, descriptors and out_f). A window outside [0, f] is clamped into it
+ * and raises the RESA_ERR_BAD_INDEX flag. Requires 1 <= f <= len_bound and
+ * f <= 256. */
 RESA_API int resa_rectify_varlen(const resa_dims* dims, const void* q_f, const void* k_f,
                                  const void* v_f, void* k_cache, void* v_cache, void* desc,
-                                 const int32_t* lens, int64_t len_bound, int32_t f,
-                                 float softmax_scale, void* out_f, void* workspace,
+                                 const int32_t* lens, const int32_t* windows, int64_t len_bound,
+                                 int32_t f, float softmax_scale, void* out_f, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error flags of the

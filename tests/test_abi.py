@@ -161,9 +161,13 @@ def test_varlen_calls_reject_invalid_arguments(resa):
     assert dense(bound=4097) == E.RESA_ERR_CAPACITY
 
     def rect(lens=FAKE, bound=100, f=32):
-        return lib.resa_rectify_varlen(dr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, lens, bound, f,
-                                       1.0, FAKE, FAKE, 1 << 30, None)
+        return lib.resa_rectify_varlen(dr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, lens, win, bound,
+                                       f, 1.0, FAKE, FAKE, 1 << 30, None)
+    win = None
     assert rect(lens=None) == E.RESA_ERR_INVALID_ARG
+    win = FAKE + 1                                  # misaligned windows
+    assert rect() == E.RESA_ERR_INVALID_ARG
+    win = None
     assert rect(f=101) == E.RESA_ERR_INVALID_ARG
     assert rect(f=0) == E.RESA_ERR_INVALID_ARG
     assert rect(bound=4097) == E.RESA_ERR_CAPACITY

@@ -98,7 +98,8 @@ class VarPair:
                   f"row {b} step {step} lse")
         return gsel
 
-    def rectify(self, f: int, scale: float = 1.0):
+    def rectify(self, f: int, scale: float = 1.0, windows=None):
+        """windows: per-row windows (None: f for every row)."""
         spec, resa = self.spec, self.resa
         q_f, k_f, v_f = rectify_inputs(spec, self.rect_calls, self.bound(), f)
         self.rect_calls += 1
@@ -106,19 +107,23 @@ class VarPair:
         out = torch.full((spec.batch, f, spec.n_q_heads, spec.head_dim), sentinel,
                          dtype=tdt(spec.dtype), device="cuda")
         before = (self.k.clone(), self.v.clone(), self.desc.clone())
+        win_t = None if windows is None else torch.tensor(windows, dtype=torch.int32,
+                                                          device="cuda")
         resa.rectify_varlen(to_dev(q_f, spec.dtype), to_dev(k_f, spec.dtype),
                             to_dev(v_f, spec.dtype), self.k, self.v, self.desc, self.lens_t(),
-                            self.bound(), f, scale, out, self.ws)
+                            self.bound(), f, scale, out, self.ws, windows=win_t)
         assert resa.workspace_status(self.ws) == resa.RESA_OK
         got = out.float().cpu().numpy()
         for b, st in enumerate(self.states):
-            if st.length < f:   # shorter than the window: left untouched
+            w = f if windows is None else int(windows[b])
+            if w == 0 or st.length < w:   # not rectified: left untouched
                 assert (got[b] == sentinel).all(), f"row {b}: output written"
                 for new, old in zip((self.k, self.v, self.desc), before):
                     assert torch.equal(new[b], old[b]), f"row {b}: cache touched"
                 continue
-            ref = st.rectify(q_f[b:b + 1], k_f[b:b + 1], v_f[b:b + 1], f, scale)
-            close(got[b], ref[0], spec.dtype, f"row {b} (len {st.length}) rectify f={f}")
+            ref = st.rectify(q_f[b:b + 1, :w], k_f[b:b + 1, :w], v_f[b:b + 1, :w], w, scale)
+            close(got[b, :w], ref[0], spec.dtype, f"row {b} (len {st.length}) rectify w={w}")
+            assert (got[b, w:] == sentinel).all(), f"row {b}: rows past its window written"
 
 
 def test_varlen_bf16_decode_and_rectify(resa):
@@ -206,6 +211,24 @@ def test_varlen_equal_lengths_match_fixed_length_call_bitwise(resa):
     resa.rectify_varlen(q_f, k_f, v_f, kb, vb, db, lens + 1, 6001, 32, 1.0, rb, wb)
     assert torch.equal(ra, rb)
     assert torch.equal(ka, kb) and torch.equal(va, vb) and torch.equal(da, db)
+
+
+def test_varlen_rectify_phases(resa):
+    """Rows at different rectification phases in one call: full window,
+    skipped (0), partial windows (1, 17, 40 of f = 48), on the tensor-core
+    path (bf16, G = 4) and on the CUDA-core path (fp32)."""
+    for dtype in ("bf16", "f32"):
+        spec = Spec(batch=5, n_q_heads=16, n_kv_heads=4, head_dim=128 if dtype == "bf16" else 64,
+                    len0=3000, steps=60, dtype=dtype, r=0.1, n_min=8, rect_block_mean=False)
+        p = VarPair(resa, spec, [3000, 2500, 1000, 45, 2222])
+        for step in range(48):
+            p.decode(step)
+        p.rectify(48, windows=[48, 0, 17, 1, 40])
+        p.desc_matches()
+        p.decode(48)
+        p.rectify(48, windows=[0, 48, 48, 0, 3])
+        p.desc_matches()
+        p.decode(49)
 
 
 def test_varlen_select_beyond_register_path(resa):
@@ -299,3 +322,9 @@ def test_varlen_out_of_range_lengths_are_clamped_and_flagged(resa):
     out_f = torch.empty(2, 16, 8, 64, dtype=dt, device="cuda")
     resa.rectify_varlen(q_f, k_f, v_f, p.k, p.v, p.desc, bad, 513, 16, 1.0, out_f, p.ws)
     assert resa.workspace_status(p.ws) == resa.RESA_ERR_BAD_INDEX
+    good = torch.tensor([513, 100], dtype=torch.int32, device="cuda")
+    bad_w = torch.tensor([17, -1], dtype=torch.int32, device="cuda")   # above f, below 0
+    resa.rectify_varlen(q_f, k_f, v_f, p.k, p.v, p.desc, good, 513, 16, 1.0, out_f, p.ws,
+                        windows=bad_w)
+    assert resa.workspace_status(p.ws) == resa.RESA_ERR_BAD_INDEX
+    assert torch.isfinite(out_f[0].float()).all()
