@@ -111,13 +111,13 @@ __device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, in
     }
   }
   if (a.S == 1) return;
-  __threadfence();
+  // arrival: one acquire-release add after the CTA barrier releases every
+  // thread's partial (cumulativity) and, for the last CTA, acquires all others'
   __syncthreads();
   int* counter = a.counters + static_cast<int64_t>(br) * a.H + g;
-  if (threadIdx.x == 0) s_last = atomicAdd(counter, 1) == a.S - 1;
+  if (threadIdx.x == 0) s_last = atomic_add_acq_rel(counter, 1) == a.S - 1;
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // last CTA: each thread merges its (head, channel) outputs over all splits.
   constexpr int NT = NW * 32;
   if (a.G * D <= 2 * NT && a.S <= 32) {
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
 
 // ---------------------------------------------------------------------- launch
 constexpr int kNW = 8;        // warps per CTA (one CTA per SM for bf16)
-constexpr int kStages = 3;    // tiles in flight per warp
+constexpr int kStages = 2;    // tiles in flight per warp (3: no faster, more shared memory)
 
 template <int D>
 static cudaError_t attend_bf16_t(const Shape& s, const AttnK& k, const AttnArgs& a,
