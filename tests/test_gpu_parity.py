@@ -156,6 +156,47 @@ def test_crowded_ties_take_lowest_indices():
         assert np.array_equal(res["gpu_sel"], res["sel"])
 
 
+@pytest.mark.parametrize("len0", [16 * 2000 + 5, 16 * 6000, 16 * 12000 + 3, 16 * 30000])
+def test_select_row_sizes(len0):
+    """Rows of 2000 to 30000 blocks: the register selection with 8 and 16 keys
+    per thread and the shared-memory one."""
+    spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, len0=len0, steps=3,
+                dtype="bf16", r=0.1, n_min=16)
+    p = Pair(spec)
+    for step in range(spec.steps):
+        p.decode(step)
+    assert p.desc_matches()
+
+
+@pytest.mark.parametrize("r,n_min", [(1.0, 16), (1e-4, 1)])
+def test_select_every_block_and_local_only(r, n_min):
+    """n = M (every block kept) and n = 1 (only the local block) on a row of
+    3000 blocks."""
+    spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, len0=16 * 3000 + 7, steps=2,
+                dtype="bf16", r=r, n_min=n_min)
+    p = Pair(spec)
+    for step in range(spec.steps):
+        res = p.decode(step)
+        M = orc.num_blocks(p.length)
+        expect = list(range(M)) if res["n"] == M else [M - 1]
+        assert res["n"] in (1, M)
+        assert [list(x) for x in res["gpu_sel"][0]] == [expect, expect]
+
+
+def test_all_tied_scores_on_a_long_row():
+    """Every block identical at 3000 blocks: the whole row ties, the lowest
+    indices are kept."""
+    spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=16 * 3000, steps=2,
+                dtype="bf16", r=0.1, n_min=4)
+    K, V = make_cache(spec)
+    K[:] = round_to(np.full_like(K, 0.5), "bf16")
+    p = Pair(spec, cache=(K, V))
+    for step in range(spec.steps):
+        res = p.decode(step)
+        n, M = res["n"], orc.num_blocks(p.length)
+        assert list(res["gpu_sel"][0, 0]) == list(range(n - 1)) + [M - 1]
+
+
 def test_select_beyond_shared_memory_keys():
     """More blocks than the selection keeps in shared memory (M > 40960)."""
     spec = Spec(batch=1, n_q_heads=4, n_kv_heads=1, head_dim=64, len0=700_001, steps=2,
