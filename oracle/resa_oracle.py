@@ -167,6 +167,41 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, sel: np.ndarray, length:
     return O, lse
 
 
+# ---------------------------------------------------------------------------
+# prefill-side step: dense causal attention of a prompt + its descriptors
+# ---------------------------------------------------------------------------
+def prefill(q: np.ndarray, K: np.ndarray, V: np.ndarray, length: int, scale: float,
+            group: int):
+    """Causal dense attention of every prompt position, and the prompt's block
+    descriptors.
+
+    The decode loop of "Rectified Sparse Attention" (pith.science review,
+    "What carries the argument") starts from a prefilled cache whose 16-token
+    blocks carry Quest min/max summaries; the rectification's dense causal
+    pass, applied to every position instead of the last f, is this attention.
+
+    q: [B, len, Hq, d]; K, V: [B, Hkv, L, d] with the prompt in slots
+    [0, length). Returns (O [B, len, Hq, d] float64, lo, hi) where lo/hi are
+    build_desc(K, length). Query i sees keys 0 .. i.
+    """
+    B, L, Hq, d = q.shape
+    assert L == length
+    O = np.empty((B, L, Hq, d), dtype=np.float64)
+    visible = np.arange(L)[None, :] <= np.arange(L)[:, None]          # [i, t]: t <= i
+    for b in range(B):
+        for h in range(Hq):
+            g = h // group
+            k = K[b, g, :L, :].astype(np.float64)
+            v = V[b, g, :L, :].astype(np.float64)
+            z = scale * (q[b, :, h, :].astype(np.float64) @ k.T)          # [i, t]
+            z = np.where(visible, z, -np.inf)
+            m = z.max(axis=1, keepdims=True)
+            p = np.exp(z - m)
+            O[b, :, h, :] = (p @ v) / p.sum(axis=1, keepdims=True)
+    lo, hi = build_desc(K, length)
+    return O, lo, hi
+
+
 class State:
     """Cache + descriptors of one sequence batch, stored in the input dtype."""
 

@@ -299,6 +299,57 @@ def test_rectify_whole_sequence_is_causal_attention():
     assert np.allclose(np.transpose(O, (0, 2, 1, 3)), ref, rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------------------- prefill
+def _prefill_case(seed, B=2, Hq=4, Hkv=2, d=8, L=80, length=53):
+    rng = np.random.default_rng(seed)
+    K = np.zeros((B, Hkv, L, d), np.float32)
+    V = np.zeros_like(K)
+    K[:, :, :length] = rng.standard_normal((B, Hkv, length, d))
+    V[:, :, :length] = rng.standard_normal((B, Hkv, length, d))
+    q = rng.standard_normal((B, length, Hq, d)).astype(np.float32)
+    return q, K, V
+
+
+@pytest.mark.parametrize("length", [1, 16, 53])
+def test_prefill_equals_causal_sdpa(length):
+    q, K, V = _prefill_case(21, length=length)
+    O, lo, hi = orc.prefill(q, K, V, length, 0.6, group=2)
+    qt = torch.from_numpy(np.transpose(q, (0, 2, 1, 3)).astype(np.float64))
+    kt = torch.from_numpy(K[:, :, :length].astype(np.float64))
+    vt = torch.from_numpy(V[:, :, :length].astype(np.float64))
+    ref = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=0.6,
+                                         enable_gqa=True).numpy()
+    assert np.allclose(np.transpose(O, (0, 2, 1, 3)), ref, rtol=0, atol=1e-12)
+    # the descriptors are the per-block min/max of the prompt's keys
+    for j in range(orc.num_blocks(length)):
+        blk = K[:, :, 16 * j:min(16 * j + 16, length)]
+        assert np.array_equal(lo[:, :, j], blk.min(axis=2))
+        assert np.array_equal(hi[:, :, j], blk.max(axis=2))
+
+
+def test_prefill_rows_are_dense_decodes():
+    """Row i of the prefill is a dense decode of query i over the first i + 1
+    tokens (another code path of the oracle)."""
+    q, K, V = _prefill_case(22, B=1, length=40)
+    O, _, _ = orc.prefill(q, K, V, 40, 0.9, group=2)
+    for i in (0, 15, 16, 39):
+        st = orc.State(K, V, i + 1, group=2)
+        Od, _ = st.dense(q[:, i], 0.9)
+        assert np.allclose(O[:, i], Od, rtol=0, atol=1e-12)
+
+
+def test_prefill_tail_is_the_rectification():
+    """The last f rows equal a rectification of the same f tokens."""
+    q, K, V = _prefill_case(23, B=1, length=50)
+    O, _, _ = orc.prefill(q, K, V, 50, 1.0, group=2)
+    st = orc.State(K, V, 50, group=2)
+    f = 18
+    k_f = np.transpose(K[:, :, 32:50], (0, 2, 1, 3)).copy()
+    v_f = np.transpose(V[:, :, 32:50], (0, 2, 1, 3)).copy()
+    Of = st.rectify(q[:, 32:50], k_f, v_f, f, 1.0)
+    assert np.allclose(O[:, 32:50], Of, rtol=0, atol=1e-12)
+
+
 # ------------------------------------------------------------ workload generator
 def test_workload_bf16_rounding_is_exact_and_nearest():
     x = np.array([1.0, 1.00390625, 1.005859375, -3.14159, 1e-3], np.float32)
@@ -371,6 +422,21 @@ def test_planted_mistakes_fail_a_pin(monkeypatch):
     def attend_drops_last_token(q, K, V, sel, length, scale, group):
         return real_attend(q, K, V, sel, length - 1, scale, group)
 
+    real_prefill = orc.prefill
+
+    def prefill_sees_next_token(q, K, V, length, scale, group):   # mask t <= i + 1
+        O, lo, hi = real_prefill(q, K, V, length, scale, group)
+        B, L, Hq, d = q.shape
+        vis = np.arange(L)[None, :] <= np.arange(L)[:, None] + 1
+        for b in range(B):
+            for h in range(Hq):
+                k = K[b, h // group, :L].astype(np.float64)
+                v = V[b, h // group, :L].astype(np.float64)
+                z = np.where(vis, scale * (q[b, :, h].astype(np.float64) @ k.T), -np.inf)
+                p = np.exp(z - z.max(axis=1, keepdims=True))
+                O[b, :, h] = (p @ v) / p.sum(axis=1, keepdims=True)
+        return O, lo, hi
+
     cases = [
         ("select_blocks", select_ties_high, test_select_all_tied_takes_lowest),
         ("select_blocks", select_drop_local, lambda: test_local_block_kept_even_if_lowest()),
@@ -378,6 +444,7 @@ def test_planted_mistakes_fail_a_pin(monkeypatch):
         ("group_scores", scores_wrong_sign, test_quest_bound_is_upper_bound),
         ("num_selected", budget_no_guard, test_num_selected_golden),
         ("attend", attend_drops_last_token, test_r1_decode_equals_sdpa_including_new_token),
+        ("prefill", prefill_sees_next_token, lambda: test_prefill_equals_causal_sdpa(53)),
     ]
     for name, bad, pin in cases:
         with monkeypatch.context() as mp:
