@@ -42,7 +42,7 @@ EXPORTED = ("resa_num_selected", "resa_workspace_bytes", "resa_build_desc",
             "resa_decode_dense", "resa_rectify",
             "resa_workspace_status", "resa_status_string", "resa_decode_sparse_noalloc",
             "resa_build_desc_varlen", "resa_decode_sparse_varlen", "resa_decode_dense_varlen",
-            "resa_rectify_varlen")
+            "resa_rectify_varlen", "resa_prefill")
 
 
 class Dims(ctypes.Structure):
@@ -93,6 +93,9 @@ _lib.resa_rectify_varlen.restype = ctypes.c_int
 _lib.resa_rectify_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P,
                                      ctypes.c_size_t, _P]
+_lib.resa_prefill.restype = ctypes.c_int
+_lib.resa_prefill.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.c_int64, ctypes.c_float,
+                              _P, _P, ctypes.c_size_t, _P]
 _lib.resa_workspace_status.restype = ctypes.c_int
 _lib.resa_workspace_status.argtypes = [_P, _P]
 _lib.resa_status_string.restype = ctypes.c_char_p
@@ -275,3 +278,13 @@ def rectify_varlen(q_f, k_f, v_f, k_cache, v_cache, desc, lens, len_bound: int, 
         ctypes.byref(dims), _ptr(q_f), _ptr(k_f), _ptr(v_f), _ptr(k_cache), _ptr(v_cache),
         _ptr(desc), _lens(lens), None if windows is None else _lens(windows), int(len_bound), int(f), float(softmax_scale), _ptr(out_f),
         _ptr(workspace), workspace.numel(), _stream(stream)), "resa_rectify_varlen")
+
+
+def prefill(q, k_cache, v_cache, desc, length: int, softmax_scale: float, out, workspace,
+            stream=None) -> None:
+    """Causal attention of every prompt position (q, out: [B, len, Hq, d]) and
+    the descriptors of the prompt's keys, in one pass."""
+    dims = dims_for(k_cache, q.shape[2])
+    _check(_lib.resa_prefill(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(desc),
+                             int(length), float(softmax_scale), _ptr(out), _ptr(workspace),
+                             workspace.numel(), _stream(stream)), "resa_prefill")

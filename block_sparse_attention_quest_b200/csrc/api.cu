@@ -525,6 +525,40 @@ int resa_rectify_varlen(const resa_dims* dims, const void* q_f, const void* k_f,
                       out_f, workspace, workspace_bytes, stream, lens, windows);
 }
 
+int resa_prefill(const resa_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                 void* desc, int64_t len, float softmax_scale, void* out, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_decode_common(dims, &s, q, nullptr, nullptr, k_cache, v_cache, len, out,
+                               workspace, workspace_bytes, 0);
+  if (rc != RESA_OK) return rc;
+  if (!desc || !aligned16(desc) || !(std::isfinite(softmax_scale) && softmax_scale > 0.f))
+    return RESA_ERR_INVALID_ARG;
+  if (!rectify_on_tensor_cores(s)) return RESA_ERR_UNSUPPORTED;   // bf16, group 1/2/4/8
+  const int64_t mt64 = (len * s.G + 127) / 128;
+  if (mt64 > 65535) return RESA_ERR_UNSUPPORTED;
+  const int mtiles = static_cast<int>(mt64);
+  if (static_cast<int64_t>(s.B) * mtiles > 65535 || len * s.B > 2147483647LL) return RESA_ERR_UNSUPPORTED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const WsLayout w = ws_layout(s, len, 0);
+  RectArgs r{};
+  r.B = s.B; r.H = s.H; r.Hq = s.Hq; r.G = s.G; r.D = s.D;
+  r.f = static_cast<int>(len);          // every position is a query row
+  r.mtiles = mtiles;
+  r.S = 1;                              // m-tiles give the parallelism: no key splits
+  r.len = len; r.L_max = s.L_max; r.scale = softmax_scale; r.out = out;
+  r.part_o = reinterpret_cast<float*>(ws + w.part_o);
+  r.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  r.ctrl = reinterpret_cast<Ctrl*>(ws);
+  r.desc = desc;
+  CUtensorMap tq, tk, tv;
+  if (!make_query_map(&tq, q, s, static_cast<int>(len)) || !make_cache_map(&tk, k_cache, s, 128) ||
+      !make_cache_map(&tv, v_cache, s, 128))
+    return RESA_ERR_CUDA;
+  r.tm_q = &tq; r.tm_k = &tk; r.tm_v = &tv;
+  return cuda_status(launch_rectify_tc(r, static_cast<cudaStream_t>(stream)));
+}
+
 int resa_workspace_status(void* workspace, void* stream) {
   if (!workspace) return RESA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

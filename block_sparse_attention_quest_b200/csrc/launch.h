@@ -108,6 +108,7 @@ struct RectArgs {
   const int32_t* lens;    // optional per-row lengths [B]
   const int32_t* windows; // optional per-row windows [B] in [0, f]; rows with window 0 or
                           // shorter than their window are skipped
+  void* desc;             // prefill (f = len, S = 1): descriptors written from the K tiles
   float scale;
   void* out;              // [B][f][Hq][D] bf16
   float* part_o;          // [B*f*Hq][S][D]

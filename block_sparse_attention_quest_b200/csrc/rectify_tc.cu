@@ -41,7 +41,9 @@ struct RectK {
   int64_t L_max;
   const int32_t* lens;   // optional per-row lengths [B] (len: their bound)
   const int32_t* windows;  // optional per-row windows [B] in [0, f]
-  int H, Hq, G, f, S, mtiles;
+  __nv_bfloat16* desc;   // prefill: descriptors of the queries' own tokens, or nullptr
+  int64_t Mmax;
+  int B, H, Hq, G, f, S, mtiles;
   float scale_log2;
 };
 
@@ -85,14 +87,21 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   auto sV = [&](int w) { return sStage + w * C::kStageBytes + C::kKBytes; };
   auto sP = [&](int w) { return sStage + w * C::kStageBytes + 2 * C::kKBytes; };
 
+  // grid z runs over (m-tile, batch row) with the m-tiles that see the most
+  // keys first
   const int s_idx = blockIdx.x, g = blockIdx.y;
-  const int b = blockIdx.z / a.mtiles, mt = blockIdx.z % a.mtiles;
+  const int b = blockIdx.z % a.B, mt = a.mtiles - 1 - static_cast<int>(blockIdx.z / a.B);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t len = row_len(a.lens, a.len, b);
   const int win = row_window(a.windows, a.f, b);   // query rows in use: 0 .. win-1
   if (win == 0 || len < win) return;       // not rectified: skipped
   if (mt * 128 >= win * a.G) return;       // this m-tile holds no row in use
-  const int n_tiles = static_cast<int>((len + 127) / 128);
+  // positions of this m-tile's first and last query rows; keys past the last
+  // are masked for every row, so their tiles are not visited
+  const int64_t qpos_lo = len - win + (mt * 128) / a.G;
+  const int rows_hi = (mt + 1) * 128 < win * a.G ? (mt + 1) * 128 : win * a.G;
+  const int64_t qpos_hi = len - win + (rows_hi - 1) / a.G;
+  const int n_tiles = static_cast<int>(qpos_hi / 128) + 1;
   const int t0 = static_cast<int>(static_cast<int64_t>(s_idx) * n_tiles / a.S);
   const int t1 = static_cast<int>(static_cast<int64_t>(s_idx + 1) * n_tiles / a.S);
   const int nt = t1 - t0;
@@ -219,7 +228,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       const int64_t key0 = static_cast<int64_t>(t0 + t) * 128;
       // keys above the smallest causal limit of the tile (or past the end of
       // the cache) exist only in the last tiles
-      const bool masked = key0 + 127 > len - win;
+      const bool masked = key0 + 127 > qpos_lo;
       const int lim = masked ? static_cast<int>(qpos - key0 < 127 ? qpos - key0 : 127) : 127;
       // pass 1: row maximum of the raw scores
       float mx = -INFINITY;
@@ -307,6 +316,38 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
     if (ok && has) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_pv[w], (u - 1) & 1, a.ctrl));
       tc::fence_after_sync();
+    }
+    // prefill: the descriptors of this m-tile's own tokens (min and max of
+    // their keys per 16-token block), read from the last key tile, which holds
+    // them and receives no further copy, so K is read from HBM only once
+    if (a.desc != nullptr && nt > 0 && s_idx == a.S - 1 && w == ((nt - 1) & 1)) {
+      const int64_t key_last = static_cast<int64_t>(t0 + nt - 1) * 128;
+      const int r0 = static_cast<int>(qpos_lo - key_last);       // its first token's row
+      const int ntok = 128 / a.G;
+      if (row < D) {
+        const uint8_t* kt = sK(w);
+        const int half = row >> 6, chunk = (row & 63) >> 3, e = row & 7;
+        const int64_t bh = static_cast<int64_t>(b) * a.H + g;
+        for (int blk = 0; blk * 16 < ntok; ++blk) {
+          const int64_t tb = qpos_lo + blk * 16;
+          if (tb >= len) break;
+          const int cnt = len - tb < 16 ? static_cast<int>(len - tb) : 16;
+          float mn = INFINITY, mx = -INFINITY;
+          for (int rr = 0; rr < cnt; ++rr) {
+            const int kr = r0 + blk * 16 + rr;
+            const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                kt + half * C::kHalfBytes + kr * 128 + ((chunk ^ (kr & 7)) << 4) + e * 2));
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+          }
+          __nv_bfloat16* d = a.desc + (bh * a.Mmax + tb / 16) * 2 * D;
+          d[row] = __float2bfloat16_rn(mn);
+          d[D + row] = __float2bfloat16_rn(mx);
+        }
+      }
+      // group 1 reuses this stage for its hand-over below: every thread of
+      // the group has read it first
+      if (w == 1) asm volatile("bar.sync 2, 128;" ::: "memory");
     }
     // combine the two warpgroups: group 1 hands (m, l, O) over through its own
     // stage's K/V memory, idle once its last PV product has completed (no
@@ -458,6 +499,7 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   k.out = r.out; k.part_o = r.part_o; k.part_ml = r.part_ml; k.ctrl = r.ctrl;
   k.len = r.len; k.L_max = r.L_max; k.H = r.H; k.Hq = r.Hq; k.G = r.G; k.f = r.f; k.S = r.S;
   k.lens = r.lens; k.windows = r.windows;
+  k.desc = static_cast<__nv_bfloat16*>(r.desc); k.Mmax = r.L_max / 16; k.B = r.B;
   k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
   dim3 grid(r.S, r.H, r.B * r.mtiles);
   rectify_tc_kernel<D><<<grid, 288, C::kSmem, st>>>(*r.tm_q, *r.tm_k, *r.tm_v, k);

@@ -199,6 +199,26 @@ RESA_API int resa_decode_sparse_noalloc(const resa_dims* dims, const void* q, co
                                         float softmax_scale, void* out, float* lse,
                                         int32_t* sel, void* stream);
 
+/* Prefill-side step: dense causal attention of every position of a prompt,
+ * with the Quest descriptors of its keys produced by the same pass ("Rectified
+ * Sparse Attention", section "What carries the argument": decoding starts from
+ * a prefilled cache whose blocks carry min/max descriptors; the causal pass is
+ * the one the rectification applies to its last f tokens, here over all of
+ * them).
+ *  - q, out: [batch][len][n_q_heads][head_dim]; k_cache, v_cache hold the
+ *    prompt's keys and values in slots [0, len) (read only);
+ *  - out[b][i][h] = softmax_t(scale * q[b][i][h] . k[b][h/G][t], t <= i) . V;
+ *  - desc receives the descriptors of blocks 0 .. ceil(len/16)-1, exactly as
+ *    resa_build_desc(len) writes them, taken from the key tiles the attention
+ *    already holds in shared memory (K is read from HBM once).
+ * bf16 and groups of 1, 2, 4 or 8 query heads only (tensor cores; other
+ * shapes return RESA_ERR_UNSUPPORTED), as do len * n_q_heads / n_kv_heads >
+ * 65535 * 128 rows. The workspace only carries the error word:
+ * resa_workspace_bytes(dims, len, 0) suffices. */
+RESA_API int resa_prefill(const resa_dims* dims, const void* q, const void* k_cache,
+                          const void* v_cache, void* desc, int64_t len, float softmax_scale,
+                          void* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- variable-length batches (continuous batching) ----
  * The pages run ReSA one sequence at a time; batching sequences of different
  * lengths is this library's extension and changes nothing per row: every row

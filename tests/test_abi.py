@@ -185,3 +185,21 @@ def test_workspace_covers_every_smaller_window(resa):
         big = resa.workspace_bytes(d, 4000, 64)
         for f in range(1, 65):
             assert resa.workspace_bytes(d, 4000, f) <= big, (kw, f)
+
+
+def test_prefill_rejects_invalid_arguments(resa):
+    E = resa
+    lib = resa._lib
+
+    def pre(d, q=FAKE, desc=FAKE, length=100, scale=1.0, ws_bytes=1 << 30):
+        return lib.resa_prefill(ctypes.byref(d), q, FAKE, FAKE, desc, length, scale, FAKE, FAKE,
+                                ws_bytes, None)
+    d = _dims(resa)
+    assert pre(d, q=None) == E.RESA_ERR_INVALID_ARG
+    assert pre(d, desc=None) == E.RESA_ERR_INVALID_ARG
+    assert pre(d, length=0) == E.RESA_ERR_INVALID_ARG
+    assert pre(d, length=4097) == E.RESA_ERR_CAPACITY
+    assert pre(d, scale=0.0) == E.RESA_ERR_INVALID_ARG
+    assert pre(d, ws_bytes=64) == E.RESA_ERR_WORKSPACE
+    assert pre(_dims(resa, dtype=resa.RESA_F32)) == E.RESA_ERR_UNSUPPORTED
+    assert pre(_dims(resa, n_q_heads=24)) == E.RESA_ERR_UNSUPPORTED      # group of 3

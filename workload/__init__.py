@@ -41,6 +41,7 @@ _S_Q, _S_KNEW, _S_VNEW = 5, 6, 7
 _S_RQ, _S_RK, _S_RV = 8, 9, 10
 _S_NEEDLE = 11
 _S_LENS = 12
+_S_PQ = 13
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -159,6 +160,15 @@ def make_cache(spec: Spec):
                 for j in pos[b, h]:
                     K[b, h, j * BLOCK:(j + 1) * BLOCK] += spec.needle_shift * qd[b, h]
     return round_to(K, spec.dtype), round_to(V, spec.dtype)
+
+
+def prefill_queries(spec: Spec) -> np.ndarray:
+    """Queries of every prompt position: [B, len0, Hq, d], N(0, 1) / sqrt(d),
+    rounded to spec.dtype (the prompt's keys and values are make_cache's)."""
+    q = _rng(spec.seed, _S_PQ).standard_normal(
+        (spec.batch, spec.len0, spec.n_q_heads, spec.head_dim), dtype=np.float32)
+    q /= np.float32(math.sqrt(spec.head_dim))
+    return round_to(q, spec.dtype)
 
 
 def length_mix(spec: Spec, min_len: int, salt: int = 0) -> np.ndarray:
