@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--r", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     return ap.parse_args()
 
 
@@ -413,11 +414,50 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if not args.no_prefill:
+        res["prefill"] = run_prefill(resa, stream, dev, tf_peak, peak_kind)
     if e2e is not None:
         res["e2e"] = {"value": round(e2e["ms_per_step"] * 1000.0 / (f * L) / world, 3),
                       "unit": "us", "h2d_bytes_per_step": e2e["h2d"],
                       "d2h_bytes_per_step": e2e["d2h"]}
     return res, spec
+
+
+def run_prefill(resa, stream, dev, tf_peak, peak_kind, length=16384):
+    """The prefill-side step (causal attention of every prompt position with
+    the descriptors from the same pass) on one prompt of `length` tokens at
+    the benchmark's head shape; CUDA events around back-to-back calls."""
+    import torch
+    from workload import Spec, prefill_queries
+    spec = Spec(batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=length, steps=0)
+    g = torch.Generator(device=dev).manual_seed(spec.seed)
+    k = torch.randn(1, 8, spec.max_len, 128, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 8, spec.max_len, 128, device=dev, generator=g).to(torch.bfloat16)
+    q = torch.from_numpy(prefill_queries(spec)).to(dev).to(torch.bfloat16)
+    desc = torch.zeros(1, 8, spec.max_blocks, 2, 128, dtype=torch.bfloat16, device=dev)
+    out = torch.empty_like(q)
+    ws = resa.alloc_workspace(resa.dims_for(k, 32), spec.max_len, 0, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            resa.prefill(q, k, v, desc, length, 1.0, out, ws)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record(stream)
+        for _ in range(reps):
+            resa.prefill(q, k, v, desc, length, 1.0, out, ws)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    assert resa.workspace_status(ws) == resa.RESA_OK
+    us = e0.elapsed_time(e1) * 1000.0 / reps
+    # QK^T and PV over the causal triangle: 4 * Hq * d * sum_i (i + 1)
+    flops = 4.0 * 32 * 128 * (length * (length + 1) / 2)
+    tflops = flops / (us * 1e-6) / 1e12
+    return {"workload": f"prefill_{length // 1024}k_b1", "us": round(us, 1),
+            "tflops": round(tflops, 1), "frac": round(tflops / tf_peak, 4),
+            "peak": tf_peak, "peak_kind": f"{peak_kind} cuBLAS bf16 (burst)",
+            "flops": flops, "bound": "tensor",
+            "note": "descriptors of the prompt written by the same pass"}
 
 
 def run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt):
