@@ -42,7 +42,7 @@ EXPORTED = ("resa_num_selected", "resa_workspace_bytes", "resa_build_desc",
             "resa_decode_dense", "resa_rectify",
             "resa_workspace_status", "resa_status_string", "resa_decode_sparse_noalloc",
             "resa_build_desc_varlen", "resa_decode_sparse_varlen", "resa_decode_dense_varlen",
-            "resa_rectify_varlen", "resa_prefill")
+            "resa_rectify_varlen", "resa_prefill", "resa_wait_check")
 
 
 class Dims(ctypes.Structure):
@@ -96,6 +96,8 @@ _lib.resa_rectify_varlen.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _
 _lib.resa_prefill.restype = ctypes.c_int
 _lib.resa_prefill.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.c_int64, ctypes.c_float,
                               _P, _P, ctypes.c_size_t, _P]
+_lib.resa_wait_check.restype = ctypes.c_int
+_lib.resa_wait_check.argtypes = [_P, ctypes.c_int32, ctypes.c_uint32, _P, _P]
 _lib.resa_workspace_status.restype = ctypes.c_int
 _lib.resa_workspace_status.argtypes = [_P, _P]
 _lib.resa_status_string.restype = ctypes.c_char_p
@@ -288,3 +290,11 @@ def prefill(q, k_cache, v_cache, desc, length: int, softmax_scale: float, out, w
     _check(_lib.resa_prefill(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(desc),
                              int(length), float(softmax_scale), _ptr(out), _ptr(workspace),
                              workspace.numel(), _stream(stream)), "resa_prefill")
+
+
+def wait_check(flag, target: int, limit_us: int, workspace, stream=None) -> None:
+    """Enqueue the device's bounded wait on `flag` (int32 CUDA tensor) reaching
+    `target`; a wait that runs out shows as RESA_ERR_TIMEOUT in
+    workspace_status()."""
+    _check(_lib.resa_wait_check(_ptr(flag), int(target), int(limit_us), _ptr(workspace),
+                                _stream(stream)), "resa_wait_check")

@@ -559,6 +559,17 @@ int resa_prefill(const resa_dims* dims, const void* q, const void* k_cache, cons
   return cuda_status(launch_rectify_tc(r, static_cast<cudaStream_t>(stream)));
 }
 
+int resa_wait_check(const int32_t* flag, int32_t target, uint32_t limit_us, void* workspace,
+                    void* stream) {
+  if (!flag || (reinterpret_cast<uintptr_t>(flag) & 3u) != 0 || !workspace ||
+      (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || limit_us < 1 ||
+      limit_us > 2000000u)
+    return RESA_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_check(flag, target, static_cast<unsigned long long>(limit_us) * 1000ull,
+                                       reinterpret_cast<Ctrl*>(workspace),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int resa_workspace_status(void* workspace, void* stream) {
   if (!workspace) return RESA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

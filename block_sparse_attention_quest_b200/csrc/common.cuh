@@ -165,6 +165,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait of one thread until *counter >= target (acquire): returns
+// false, with the time-out bit raised, once limit_ns of %globaltimer pass.
+__device__ __forceinline__ bool wait_count_bounded(const int* counter, int target,
+                                                   unsigned long long limit_ns, Ctrl* ctrl) {
+  if (ld_acquire(counter) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (ld_acquire(counter) < target) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      raise_error(ctrl, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // TMA 2-D tiled load global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {

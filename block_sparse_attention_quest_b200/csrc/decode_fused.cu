@@ -68,11 +68,7 @@ __device__ __forceinline__ uint32_t fkey(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
+
 
 // exclusive scan of one value per thread over the CTA (kFThreads threads)
 __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t x, uint32_t* wtot, uint32_t* total) {
@@ -287,14 +283,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
     __syncthreads();
     if (tid == 0) {
       atomicAdd(bar_cnt, 1);
-      const unsigned long long t0 = globaltimer_ns();
-      while (ld_acquire(bar_cnt) < a.cpg) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          raise_error(a.ctrl, kErrTimeout);
-          s_mode = -1;
-          break;
-        }
-      }
+      if (!wait_count_bounded(bar_cnt, a.cpg, kWaitLimitNs, a.ctrl)) s_mode = -1;
       __threadfence();
     }
     __syncthreads();

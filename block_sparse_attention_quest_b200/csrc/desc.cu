@@ -201,4 +201,17 @@ cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_
   return cudaGetLastError();
 }
 
+// Failure-detection check: one thread runs the bounded counter wait of the
+// one-launch decode kernel's group barrier on a caller's flag.
+__global__ void wait_check_kernel(const int* flag, int target, unsigned long long limit_ns,
+                                  Ctrl* ctrl) {
+  if (threadIdx.x == 0) (void)wait_count_bounded(flag, target, limit_ns, ctrl);
+}
+
+cudaError_t launch_wait_check(const int* flag, int target, unsigned long long limit_ns,
+                              Ctrl* ctrl, cudaStream_t st) {
+  wait_check_kernel<<<1, 32, 0, st>>>(flag, target, limit_ns, ctrl);
+  return cudaGetLastError();
+}
+
 }  // namespace resa

@@ -121,6 +121,10 @@ struct RectArgs {
 cudaError_t launch_rectify_tc(const RectArgs& r, cudaStream_t st);
 int attend_ctas_per_sm(const Shape& s);
 
+// bounded wait of one thread until *flag >= target (failure-detection check)
+cudaError_t launch_wait_check(const int* flag, int target, unsigned long long limit_ns,
+                              Ctrl* ctrl, cudaStream_t st);
+
 constexpr int kMaxSplits = 64;
 
 // Bytes at the start of a workspace that must be zero before a call (the

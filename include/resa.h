@@ -276,6 +276,18 @@ RESA_API int resa_rectify_varlen(const resa_dims* dims, const void* q_f, const v
                                  int32_t f, float softmax_scale, void* out_f, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* Failure-detection check of the device-side bounded wait (no counterpart in
+ * the method): one thread waits until the device int32 *flag >= target, as
+ * the one-launch decode kernel's group barrier waits on its arrival counter,
+ * for at most limit_us microseconds (1 .. 2,000,000). A wait that runs out
+ * sets the RESA_ERR_TIMEOUT flag of `workspace` (read by
+ * resa_workspace_status()) and the kernel returns: the context stays usable.
+ * Passing a flag that nothing sets checks that a stuck wait ends and is
+ * reported. flag: 4-byte aligned device pointer; workspace: as for the other
+ * calls. Only enqueues work on `stream`. */
+RESA_API int resa_wait_check(const int32_t* flag, int32_t target, uint32_t limit_us,
+                             void* workspace, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error flags of the
  * workspace control block. Returns RESA_OK, RESA_ERR_TIMEOUT,
  * RESA_ERR_BAD_INDEX or RESA_ERR_CUDA. */

@@ -203,3 +203,13 @@ def test_prefill_rejects_invalid_arguments(resa):
     assert pre(d, ws_bytes=64) == E.RESA_ERR_WORKSPACE
     assert pre(_dims(resa, dtype=resa.RESA_F32)) == E.RESA_ERR_UNSUPPORTED
     assert pre(_dims(resa, n_q_heads=24)) == E.RESA_ERR_UNSUPPORTED      # group of 3
+
+
+def test_wait_check_rejects_invalid_arguments(resa):
+    lib = resa._lib
+    E = resa
+    assert lib.resa_wait_check(None, 1, 1000, FAKE, None) == E.RESA_ERR_INVALID_ARG
+    assert lib.resa_wait_check(FAKE + 2, 1, 1000, FAKE, None) == E.RESA_ERR_INVALID_ARG
+    assert lib.resa_wait_check(FAKE, 1, 1000, FAKE + 16, None) == E.RESA_ERR_INVALID_ARG
+    assert lib.resa_wait_check(FAKE, 1, 0, FAKE, None) == E.RESA_ERR_INVALID_ARG
+    assert lib.resa_wait_check(FAKE, 1, 2000001, FAKE, None) == E.RESA_ERR_INVALID_ARG
