@@ -9,17 +9,19 @@
 //
 // One CTA per (KV split, KV head, batch x 128-row tile); 9 warps:
 //   warps 0-3 and 4-7  two softmax warpgroups; group w takes the key tiles
-//              t = w (mod 2) with its own S and O accumulators in TMEM and
-//              its own shared-memory stage (K, V, P), so one group's softmax
-//              overlaps the other group's MMAs. One query row per thread
-//              (= TMEM lane): row maximum, causal mask on the tail tiles only,
-//              P = 2^(s * scale - m) written bf16 to shared memory, O rescaled
-//              in TMEM only when the running maximum grows by more than 2^8;
-//              the two groups' (m, l, O) are merged at the end;
+//              t = w (mod 2) with its own S and O accumulators in TMEM, so one
+//              group's softmax overlaps the other group's MMAs. One query row
+//              per thread (= TMEM lane): row maximum, causal mask on the tiles
+//              that cross it only, P = 2^(s * scale - m) written as bf16 pairs
+//              into tensor memory over the S columns it was computed from (the
+//              A operand of the PV product), O rescaled in TMEM only when the
+//              running maximum grows by more than 2^8; the two groups'
+//              (m, l, O) are merged at the end;
 //   warp 8     one thread issues the TMA copies (Q once; K and V of each tile
-//              on separate barriers, so K of tile t+2 loads while tile t is
-//              still in its softmax) and the tcgen05.mma instructions, with
-//              completion signalled by tcgen05.commit on mbarriers.
+//              into a ring of three shared-memory stages, K and V on separate
+//              barriers so the next keys stream in while a tile is in its
+//              softmax) and the tcgen05.mma instructions, with completion
+//              signalled by tcgen05.commit on mbarriers.
 // The row order inside a tile is m = i * G + h (query i of head h of the
 // group), which is exactly the layout of q_f[b][i][g*G + h][:] viewed as a
 // 3-D tensor, so Q arrives by one box per 64-channel half.
@@ -53,11 +55,10 @@ struct RectCfg {
   static constexpr int kHalfBytes = 128 * 128;            // [128 rows][64 bf16]
   static constexpr int kQBytes = kHalves * kHalfBytes;
   static constexpr int kKBytes = kHalves * kHalfBytes;    // K (or V) of one 128-key tile
-  static constexpr int kPBytes = 2 * kHalfBytes;          // [128 rows][128 keys]
-  // two stages, one per softmax warpgroup: stage w holds K, V and P of the
-  // tiles t = w (mod 2)
-  static constexpr int kStageBytes = 2 * kKBytes + kPBytes;
-  static constexpr int kSmem = kQBytes + 2 * kStageBytes + 1024;
+  // K/V ring: tile t uses stage t % kStages (P lives in tensor memory)
+  static constexpr int kStages = 3;
+  static constexpr int kStageBytes = 2 * kKBytes;
+  static constexpr int kSmem = kQBytes + kStages * kStageBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;              // S0 S1 O0 O1, 128 columns each
 };
 
@@ -75,7 +76,8 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   using C = RectCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q;
-  __shared__ __align__(8) uint64_t bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
+  __shared__ __align__(8) uint64_t bar_kfull[C::kStages], bar_kempty[C::kStages];
+  __shared__ __align__(8) uint64_t bar_vfull[C::kStages], bar_vempty[C::kStages];
   __shared__ __align__(8) uint64_t bar_s[2], bar_p[2], bar_pv[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ float s_m1[128], s_l1[128];
@@ -83,9 +85,8 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = base;
   uint8_t* sStage = sQ + C::kQBytes;
-  auto sK = [&](int w) { return sStage + w * C::kStageBytes; };
-  auto sV = [&](int w) { return sStage + w * C::kStageBytes + C::kKBytes; };
-  auto sP = [&](int w) { return sStage + w * C::kStageBytes + 2 * C::kKBytes; };
+  auto sK = [&](int st) { return sStage + st * C::kStageBytes; };
+  auto sV = [&](int st) { return sStage + st * C::kStageBytes + C::kKBytes; };
 
   // grid z runs over (m-tile, batch row) with the m-tiles that see the most
   // keys first
@@ -109,11 +110,14 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
 #pragma unroll
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(&bar_kfull[st], 1);
+      mbar_init(&bar_kempty[st], 1);
+      mbar_init(&bar_vfull[st], 1);
+      mbar_init(&bar_vempty[st], 1);
+    }
+#pragma unroll
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&bar_kfull[w], 1);
-      mbar_init(&bar_kempty[w], 1);
-      mbar_init(&bar_vfull[w], 1);
-      mbar_init(&bar_vempty[w], 1);
       mbar_init(&bar_s[w], 1);
       mbar_init(&bar_p[w], 128);
       mbar_init(&bar_pv[w], 1);
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf) tma_load_2d(dst + hf * C::kHalfBytes, map, hf * 64, y, bar);
       };
-      for (int t = 0; t < nt && t < 2; ++t) {
+      for (int t = 0; t < nt && t < C::kStages; ++t) {
         load(&tmK, sK(t), &bar_kfull[t], t);
         load(&tmV, sV(t), &bar_vfull[t], t);
       }
@@ -155,8 +159,8 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       constexpr uint32_t idO = tc::idesc_bf16(128, D, true);
       const uint32_t q_addr = smem_u32(sQ);
       auto issue_qk = [&](int t) {
-        const int w = t & 1;
-        const uint32_t k_addr = smem_u32(sK(w));
+        const int w = t & 1, st = t % C::kStages;
+        const uint32_t k_addr = smem_u32(sK(st));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
@@ -164,20 +168,19 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
                      tc::smem_desc(k_addr + off, 16, 1024), idS, kk > 0);
         }
         tc::commit(&bar_s[w]);
-        tc::commit(&bar_kempty[w]);
+        tc::commit(&bar_kempty[st]);
       };
+      // P of tile t sits in tensor memory over S of its group: 16 keys per
+      // k-step = 8 columns of bf16 pairs
       auto issue_pv = [&](int t) {
-        const int w = t & 1;
-        const uint32_t v_addr = smem_u32(sV(w));
-        const uint32_t p_addr = smem_u32(sP(w));
+        const int w = t & 1, st = t % C::kStages;
+        const uint32_t v_addr = smem_u32(sV(st));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t poff = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc::mma_ss(tO(w), tc::smem_desc(p_addr + poff, 16, 1024),
-                     tc::smem_desc(v_addr + kk * 2048, C::kHalfBytes, 1024), idO, t >= 2 || kk > 0);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_ts(tO(w), tS(w) + 8u * kk, tc::smem_desc(v_addr + kk * 2048, C::kHalfBytes, 1024),
+                     idO, t >= 2 || kk > 0);
         tc::commit(&bar_pv[w]);
-        tc::commit(&bar_vempty[w]);
+        tc::commit(&bar_vempty[st]);
       };
       bool ok = mbar_wait_bounded(&bar_q, 0, a.ctrl);
       for (int t = 0; ok && t < nt && t < 2; ++t) {
@@ -187,22 +190,25 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
         issue_qk(t);
       }
       for (int t = 0; ok && t < nt; ++t) {
-        const int w = t & 1;
-        const uint32_t ph = (t >> 1) & 1;
-        const bool refill = t + 2 < nt;
+        const int w = t & 1, st = t % C::kStages;
+        const uint32_t ph = (t / C::kStages) & 1;      // phase of stage st for tile t
+        const bool refill = t + C::kStages < nt;
         // K of tile t is no longer needed once QK(t) completed
         if (refill) {
-          if (!(ok = mbar_wait_bounded(&bar_kempty[w], ph, a.ctrl))) break;
-          load(&tmK, sK(w), &bar_kfull[w], t + 2);
+          if (!(ok = mbar_wait_bounded(&bar_kempty[st], ph, a.ctrl))) break;
+          load(&tmK, sK(st), &bar_kfull[st], t + C::kStages);
         }
-        if (!(ok = mbar_wait_bounded(&bar_p[w], ph, a.ctrl))) break;
-        if (!(ok = mbar_wait_bounded(&bar_vfull[w], ph, a.ctrl))) break;
+        if (!(ok = mbar_wait_bounded(&bar_p[w], (t >> 1) & 1, a.ctrl))) break;
+        if (!(ok = mbar_wait_bounded(&bar_vfull[st], ph, a.ctrl))) break;
         tc::fence_after_sync();
         issue_pv(t);
-        if (refill) {
-          if (!(ok = mbar_wait_bounded(&bar_vempty[w], ph, a.ctrl))) break;
-          load(&tmV, sV(w), &bar_vfull[w], t + 2);
-          if (!(ok = mbar_wait_bounded(&bar_kfull[w], ph ^ 1, a.ctrl))) break;
+        // PV(t) reads P from this group's S columns, which QK(t + 2) rewrites:
+        // it is issued only once PV(t) has completed
+        if (!(ok = mbar_wait_bounded(&bar_vempty[st], ph, a.ctrl))) break;
+        if (refill) load(&tmV, sV(st), &bar_vfull[st], t + C::kStages);
+        if (t + 2 < nt) {
+          const int st2 = (t + 2) % C::kStages;
+          if (!(ok = mbar_wait_bounded(&bar_kfull[st2], ((t + 2) / C::kStages) & 1, a.ctrl))) break;
           tc::fence_after_sync();
           issue_qk(t + 2);
         }
@@ -267,41 +273,38 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
         l *= alpha;
         m_ref = m_new;
       }
-      // pass 2: P = 2^(s * scale - m_ref) as bf16 (K-major, 128-byte swizzle)
+      // pass 2: P = 2^(s * scale - m_ref) as bf16 pairs into TMEM columns
+      // 16 c4 .. 16 c4 + 15 of S (keys 32 c4 .. 32 c4 + 31): below the columns
+      // still to be read, above none the A operand needs later
       const bool live = m_ref != -INFINITY;
       float sum = 0.f;
-      uint8_t* pw = sP(w);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         float v[32];
         tc::ld32(tS(w) + lane_off + c4 * 32, v);
         tc::wait_ld();
+        uint32_t wd[16];
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t wd[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = c4 * 32 + c8 * 8 + 2 * e;
-            float p0 = ex2(fmaf(v[c8 * 8 + 2 * e], sl2, -m_ref));
-            float p1 = ex2(fmaf(v[c8 * 8 + 2 * e + 1], sl2, -m_ref));
-            if (masked) {
-              if (c > lim) p0 = 0.f;
-              if (c + 1 > lim) p1 = 0.f;
-            }
-            if (!live) { p0 = 0.f; p1 = 0.f; }
-            sum += p0 + p1;
-            wd[e] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 16; ++e) {
+          const int c = c4 * 32 + 2 * e;
+          float p0 = ex2(fmaf(v[2 * e], sl2, -m_ref));
+          float p1 = ex2(fmaf(v[2 * e + 1], sl2, -m_ref));
+          if (masked) {
+            if (c > lim) p0 = 0.f;
+            if (c + 1 > lim) p1 = 0.f;
           }
-          const int chunk = c4 * 4 + c8;                   // 16-byte chunk of 8 keys
-          uint8_t* dst = pw + (chunk >> 3) * C::kHalfBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          if (!live) { p0 = 0.f; p1 = 0.f; }
+          sum += p0 + p1;
+          wd[e] = pack_bf16x2(p0, p1);
         }
+        tc::st16(tS(w) + lane_off + c4 * 16, wd);
       }
+      tc::wait_st();
       l += sum;
       // V rows past the end of the cache are zeroed (0 * stale data must not
       // reach an output)
       if (key0 + row >= len) {
-        uint8_t* v = sV(w);
+        uint8_t* v = sV(t % C::kStages);
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf)
 #pragma unroll
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       const int r0 = static_cast<int>(qpos_lo - key_last);       // its first token's row
       const int ntok = 128 / a.G;
       if (row < D) {
-        const uint8_t* kt = sK(w);
+        const uint8_t* kt = sK((nt - 1) % C::kStages);
         const int half = row >> 6, chunk = (row & 63) >> 3, e = row & 7;
         const int64_t bh = static_cast<int64_t>(b) * a.H + g;
         for (int blk = 0; blk * 16 < ntok; ++blk) {
@@ -349,10 +352,13 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       // the group has read it first
       if (w == 1) asm volatile("bar.sync 2, 128;" ::: "memory");
     }
-    // combine the two warpgroups: group 1 hands (m, l, O) over through its own
-    // stage's K/V memory, idle once its last PV product has completed (no
-    // copy targets that stage after group 1's last tile)
-    float* sO1 = reinterpret_cast<float*>(sK(1));            // [128][D], 64 KB at most
+    // combine the two warpgroups: group 1 hands (m, l, O) over through the
+    // K/V stage of its last tile, idle once that tile's PV product has
+    // completed (no copy targets it afterwards, and group 0's remaining tile
+    // uses another stage); with no tile of its own, through stage 1, which
+    // is never loaded then
+    const int t_last1 = (nt & 1) ? nt - 2 : nt - 1;          // last odd tile
+    float* sO1 = reinterpret_cast<float*>(sK(nt >= 2 ? t_last1 % C::kStages : 1));
     if (w == 1) {
       s_m1[row] = has ? m_ref : -INFINITY;
       s_l1[row] = has ? l : 0.f;
