@@ -250,6 +250,9 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
 
+  // the next kernel in the stream may start its prologue now (whatever it
+  // reads from this kernel it reads after its own dependency wait)
+  grid_launch_dependents();
   const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
   const int b = br / a.R, r = br % a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -451,6 +454,7 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
   extern __shared__ float smf[];
   float* sq = smf;                            // [8][D]
   float* tiles = smf + 8 * D;                 // [NW][2][16][P]
+  grid_launch_dependents();
   const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
   const int b = br / a.R, r = br % a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -94,6 +94,10 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   constexpr int NW = 8;
 
   __shared__ float coef[2 * D];                    // [N (for lo) | P (for hi)]
+  // launched as a programmatic dependent of whatever precedes it in the
+  // stream (q, the cache and the descriptors may come from there): nothing is
+  // read before the wait, only the launch overlaps the previous kernel's tail
+  grid_dependency_wait();
   grid_launch_dependents();
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -218,8 +222,16 @@ static cudaError_t score_t(const Shape& s, const ScoreArgs& a0, int num_sms, cud
   a.blocks_per_cta = bpc;
   const int chunks = max(1, (scored + bpc - 1) / bpc);
   dim3 grid(chunks, s.H, s.B);
-  score_kernel<T, D><<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_kernel<T, D>, a);
 }
 
 cudaError_t launch_score(const Shape& s, const void* q, const void* desc, float* scores,
