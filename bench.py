@@ -461,40 +461,61 @@ def run_prefill(resa, stream, dev, tf_peak, peak_kind, length=16384):
 
 
 def run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt):
-    """The same step through the public calls, with every step's inputs copied
-    from pinned host memory and every output copied back, inside the timed
-    region."""
+    """The same step through the public calls with host buffers: every step
+    copies its inputs (each decode call's q, k_new, v_new for every layer and
+    position, and each layer's rectify inputs) from one pinned host buffer to
+    the device, runs the calls eagerly, and reads all of the step's outputs
+    back into pinned host memory, inside the timed region."""
     import torch
     f, L = spec.f, len(layers)
     B, Hq, H, d = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
-    h_dec = [tuple(x.cpu().pin_memory() for x in s) for s in dec_in]
-    h_rect = tuple(x.cpu().pin_memory() for x in rect_in)
-    d_dec = [tuple(torch.empty_like(x) for x in s) for s in dec_in]
-    d_rect = tuple(torch.empty_like(x) for x in rect_in)
-    out = torch.empty(B, Hq, d, dtype=tdt, device=dev)
-    out_f = torch.empty(B, f, Hq, d, dtype=tdt, device=dev)
-    h_out = torch.empty(L, f, B, Hq, d, dtype=tdt).pin_memory()
-    h_out_f = torch.empty(L, B, f, Hq, d, dtype=tdt).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for s in h_dec for x in s) * L + \
-        sum(x.numel() * x.element_size() for x in h_rect) * L
-    d2h = h_out.numel() * h_out.element_size() + h_out_f.numel() * h_out_f.element_size()
+    esz = torch.empty(0, dtype=tdt).element_size()
+
+    def nbytes(x):
+        return x.numel() * x.element_size()
+
+    # packed input layout: [position][layer][q | k_new | v_new], then
+    # [layer][q_f | k_f | v_f]; every piece starts 16-byte aligned
+    pieces = [s for _ in range(1) for t in range(f) for _li in range(L) for s in dec_in[t]]
+    pieces += [x for _li in range(L) for x in rect_in]
+    offs, off = [], 0
+    for x in pieces:
+        offs.append(off)
+        off += (nbytes(x) + 15) // 16 * 16
+    h_in = torch.empty(off, dtype=torch.uint8).pin_memory()
+    for x, o in zip(pieces, offs):
+        h_in[o:o + nbytes(x)].copy_(x.cpu().contiguous().view(-1).view(torch.uint8))
+    d_in = torch.empty(off, dtype=torch.uint8, device=dev)
+
+    def view(o, like):
+        return d_in[o:o + nbytes(like)].view(tdt).view(like.shape)
+    it = iter(zip(pieces, offs))
+    d_dec = [[tuple(view(o, x) for x, o in (next(it), next(it), next(it))) for _li in range(L)]
+             for _t in range(f)]
+    d_rect = [tuple(view(o, x) for x, o in (next(it), next(it), next(it))) for _li in range(L)]
+    # every call writes its own slice of one output buffer, read back once
+    n_out = L * f * B * Hq * d
+    n_out_f = L * B * f * Hq * d
+    d_out = torch.empty(n_out + n_out_f, dtype=tdt, device=dev)
+    h_out = torch.empty(n_out + n_out_f, dtype=tdt).pin_memory()
+    out = d_out[:n_out].view(L, f, B, Hq, d)
+    out_f = d_out[n_out:].view(L, B, f, Hq, d)
+    h2d = off
+    d2h = nbytes(h_out)
 
     def step():
+        d_in.copy_(h_in, non_blocking=True)
         for t in range(f):
             length = len_start + t + 1
             for li, ly in enumerate(layers):
-                for hx, dx in zip(h_dec[t], d_dec[t]):
-                    dx.copy_(hx, non_blocking=True)
-                q, kn, vn = d_dec[t]
+                q, kn, vn = d_dec[t][li]
                 resa.decode_sparse(q, kn, vn, ly["k"], ly["v"], ly["desc"], length, spec.r,
-                                   spec.n_min, 1.0, out, ws[li])
-                h_out[li, t].copy_(out, non_blocking=True)
+                                   spec.n_min, 1.0, out[li, t], ws[li])
         for li, ly in enumerate(layers):
-            for hx, dx in zip(h_rect, d_rect):
-                dx.copy_(hx, non_blocking=True)
-            resa.rectify(d_rect[0], d_rect[1], d_rect[2], ly["k"], ly["v"], ly["desc"],
-                         len_start + f, f, 1.0, out_f, ws[li])
-            h_out_f[li].copy_(out_f, non_blocking=True)
+            q_f, k_f, v_f = d_rect[li]
+            resa.rectify(q_f, k_f, v_f, ly["k"], ly["v"], ly["desc"], len_start + f, f, 1.0,
+                         out_f[li], ws[li])
+        h_out.copy_(d_out, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(max(1, args.warmup)):
