@@ -310,6 +310,41 @@ def run_ours(args, rank, world, local_rank):
                 sel_us.append(e0.elapsed_time(e1) * 1000.0)
                 att_us.append(e1.elapsed_time(e2) * 1000.0)
 
+    # the sparse decode calls alone and the dense (r = 1) arm, each as f * L
+    # calls back to back in one CUDA graph: the method's gain over dense
+    # attention at the same length
+    def graph_us(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for t in range(f):
+                for li, ly in enumerate(layers):
+                    fn(t, li, ly)
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = 3
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1000.0 / (reps * f * L)
+
+    def sparse_call(t, li, ly):
+        q, kn, vn = dec_in[t]
+        resa.decode_sparse(q, kn, vn, ly["k"], ly["v"], ly["desc"], len_start + t + 1, spec.r,
+                           spec.n_min, 1.0, outs[li], ws[li], lse=lses[li], sel=sels[li][t])
+
+    def dense_call(t, li, ly):
+        q, kn, vn = dec_in[t]
+        resa.decode_dense(q, kn, vn, ly["k"], ly["v"], ly["desc"], len_start + t + 1, 1.0,
+                          outs[li], ws[li], lse=lses[li])
+    sparse_graph_us = graph_us(sparse_call)
+    dense_graph_us = graph_us(dense_call)
+
     # the attention kernel on its own: f * L launches back to back (every
     # layer's selected blocks, so consecutive launches read different caches)
     graph_a = torch.cuda.CUDAGraph()
@@ -386,6 +421,11 @@ def run_ours(args, rank, world, local_rank):
             "timing": "CUDA graph replay, CUDA events on the launching stream",
         },
         "decode_us": round(decode_med, 3),
+        "decode_us_p10_p90": [round(float(np.percentile(dec_us, 10)), 3),
+                              round(float(np.percentile(dec_us, 90)), 3)],
+        "sparse_decode_graph_us": round(sparse_graph_us, 3),
+        "dense_decode_graph_us": round(dense_graph_us, 3),
+        "speedup_vs_dense": round(dense_graph_us / sparse_graph_us, 2),
         "decode_kernels": "score_kernel -> select_reg_kernel -> attend_bf16_kernel (PDL chain)",
         "staged_decode_us": round(staged_med, 3),
         "staged_select_us": round(sel_med, 3),
