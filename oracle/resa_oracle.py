@@ -25,7 +25,7 @@ Sources (all from the pages describing Rectified Sparse Attention, arXiv
   schedule, the oracle computes the unsplit softmax it must equal) and Quest
   (the min/max descriptor bound).
 
-Readings where the pages are silent (each is stated again in the design doc):
+Readings where the pages are silent:
 
 * the Quest group score is sum over the group's heads h and channels c of
   max(q_hc * lo_c, q_hc * hi_c);
