@@ -213,3 +213,10 @@ def test_wait_check_rejects_invalid_arguments(resa):
     assert lib.resa_wait_check(FAKE, 1, 1000, FAKE + 16, None) == E.RESA_ERR_INVALID_ARG
     assert lib.resa_wait_check(FAKE, 1, 0, FAKE, None) == E.RESA_ERR_INVALID_ARG
     assert lib.resa_wait_check(FAKE, 1, 2000001, FAKE, None) == E.RESA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_more_blocks_than_the_selection_takes(resa):
+    """262145 blocks (4M + 16 tokens) is one block past the selection's limit:
+    rejected on the host before anything is launched."""
+    d = _dims(resa, n_q_heads=4, n_kv_heads=1, max_len=16 * 262145)
+    assert _decode(resa, d, length=16 * 262144 + 1, ws_bytes=1 << 40) == resa.RESA_ERR_UNSUPPORTED

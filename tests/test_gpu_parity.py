@@ -206,6 +206,16 @@ def test_select_beyond_shared_memory_keys():
         p.decode(step)
 
 
+def test_select_at_the_block_limit():
+    """262144 blocks (4,194,299 tokens after the step), the largest row the
+    selection accepts: keys re-read from L2 by the general radix kernel."""
+    spec = Spec(batch=1, n_q_heads=4, n_kv_heads=1, head_dim=64, len0=16 * 262144 - 6, steps=1,
+                dtype="bf16", r=0.05, n_min=16)
+    p = Pair(spec)
+    res = p.decode(0)
+    assert orc.num_blocks(p.length) == 262144 and res["n"] == 13108
+
+
 @pytest.mark.parametrize("length,f", [(100, 32), (64, 16), (48, 48), (1000, 7), (1000, 64)])
 def test_rectify_shapes(length, f):
     for dtype in ("bf16", "f32"):
