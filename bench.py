@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--workload", default="128k", choices=sorted(WORKLOADS))
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--r", type=float, default=None)
+    ap.add_argument("--f", type=int, default=None, help="rectification period (default 32)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
@@ -145,6 +146,8 @@ def run_ours(args, rank, world, local_rank):
     over = {"steps": 64}
     if args.r is not None:
         over["r"] = args.r
+    if args.f is not None:
+        over["f"] = args.f
     spec = config(cfg_idx, **over)
     f, L = spec.f, args.layers
     tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
@@ -426,6 +429,7 @@ def run_ours(args, rank, world, local_rank):
         "sparse_decode_graph_us": round(sparse_graph_us, 3),
         "dense_decode_graph_us": round(dense_graph_us, 3),
         "speedup_vs_dense": round(dense_graph_us / sparse_graph_us, 2),
+        "amortised_speedup_vs_dense": round(dense_graph_us / us_per_decode, 2),
         "decode_kernels": "score_kernel -> select_reg_kernel -> attend_bf16_kernel (PDL chain)",
         "staged_decode_us": round(staged_med, 3),
         "staged_select_us": round(sel_med, 3),
@@ -446,7 +450,8 @@ def run_ours(args, rank, world, local_rank):
             "timing": "average over f * layers back-to-back launches in one CUDA graph",
             "bound": "hbm", "achieved": round(att_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
             "frac": round(att_gbs / hbm_peak, 4),
-            "traffic": NCU_TRAFFIC.get(WORKLOAD_NAMES[cfg_idx]) if args.r is None else None,
+            "traffic": (NCU_TRAFFIC.get(WORKLOAD_NAMES[cfg_idx])
+                        if args.r is None and args.f is None else None),
             "peak_kind": f"{peak_kind} copy bandwidth",
             "bytes_per_launch": attend_bytes,
             "bytes": "selected K/V + q + out + block ids",
@@ -626,6 +631,8 @@ def run_reference(args, rank, world):
     over = {"steps": 64}
     if args.r is not None:
         over["r"] = args.r
+    if args.f is not None:
+        over["f"] = args.f
     spec = config(cfg_idx, **over)
     if rank != 0:
         return None
