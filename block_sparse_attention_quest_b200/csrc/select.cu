@@ -322,6 +322,39 @@ __device__ __forceinline__ uint32_t warp_exclusive_offset(uint32_t x, uint32_t* 
   return r;
 }
 
+// The threshold bin's c members (any order) ranked by key descending, then
+// index ascending: the member of rank take - 1 is the last one kept (the cut).
+// One warp per member, its lanes comparing it with 32 members at a time, so a
+// member costs c / 32 ballots rather than c dependent shared-memory reads.
+// Indices are distinct, so ranks are too and exactly one member writes the cut.
+__device__ __forceinline__ void rank_cut(const uint32_t* cand_rel, const int* cand_j, int c,
+                                         uint32_t take, uint32_t* cut_rel, int* cut_j) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int i = warp; i < c; i += nw) {
+    const uint32_t r = cand_rel[i];
+    const int j = cand_j[i];
+    uint32_t rank = 0;
+    for (int k0 = 0; k0 < c; k0 += 32) {
+      const int k = k0 + lane;
+      bool better = false;
+      if (k < c) {
+        const uint32_t rk = cand_rel[k];
+        better = rk > r || (rk == r && cand_j[k] < j);
+      }
+      rank += __popc(__ballot_sync(0xffffffffu, better));
+    }
+    if (lane == 0 && rank + 1 == take) {
+      *cut_rel = r;
+      *cut_j = j;
+    }
+  }
+}
+
+// kept: at or above the cut in (key descending, index ascending) order
+__device__ __forceinline__ bool at_or_above(uint32_t rel, int j, uint32_t cut_rel, int cut_j) {
+  return rel > cut_rel || (rel == cut_rel && j <= cut_j);
+}
+
 // Per-row budget for variable lengths: the row's own block count M and
 // Eq. 5 budget n (both at most the shared ones); the list keeps the shared
 // stride and its unused tail is set to -1.
@@ -348,7 +381,7 @@ __device__ __forceinline__ void row_budget(const SelRows& rl, int b, int& M, int
 // (starting at the highest bit in which the keys differ, so the bins spread
 // even when all scores share sign and exponent) locates the threshold bin;
 // its few candidates are then ranked exactly (key descending, index
-// ascending). When the bin is crowded (near-constant scores) 8-bit radix
+// ascending) to find the last one kept. When the bin is crowded (near-constant scores) 8-bit radix
 // passes continue on the remaining bits instead. The ascending output is
 // written by warps that each own a contiguous index range and order their
 // lanes with ballots, so every shared-memory read is conflict-free.
@@ -356,14 +389,15 @@ template <bool IN_SMEM>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __restrict__ scores,
                                                              int32_t* __restrict__ sel, int H,
                                                              int M, int n, SelRows rl) {
-  extern __shared__ uint32_t dyn[];               // [keys (if in smem)][chosen bitmap]
+  extern __shared__ uint32_t dyn[];               // keys (if kept in shared memory)
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t cand_rel[kCand];
   __shared__ int cand_j[kCand];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t red_min[32], red_max[32];
-  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand;
+  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand, s_cut_rel;
   __shared__ int s_mode;                          // 0 exact threshold, 1 bin floor, 2 ranked bin
+  __shared__ int s_cut_j;
   grid_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
@@ -373,8 +407,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   const int Mo = M - 1;                            // candidates: blocks 0 .. M-2
   const int need = n - 1;                          // how many of them to keep
   uint32_t* skeys = dyn;
-  uint32_t* chosen = dyn + (IN_SMEM ? M : 0);
-  const int nwords = (Mo + 31) >> 5;
 
   if (need >= Mo) {                                // every block is selected
     for (int j = tid; j < M; j += blockDim.x) out[j] = j;
@@ -408,7 +440,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
       }
     }
   }
-  for (int w = tid; w < nwords; w += blockDim.x) chosen[w] = 0u;
   for (int b = tid; b < kBins; b += blockDim.x) hist[b] = 0u;
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
@@ -467,18 +498,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
         }
       }
       __syncthreads();
-      const int c = static_cast<int>(s_ncand);
-      const uint32_t take = s_remaining;
-      for (int i = tid; i < c; i += blockDim.x) {
-        const uint32_t r = cand_rel[i];
-        const int jj = cand_j[i];
-        uint32_t rank = 0;
-        for (int k = 0; k < c; ++k) {
-          const uint32_t rk = cand_rel[k];
-          rank += (rk > r) || (rk == r && cand_j[k] < jj);
-        }
-        if (rank < take) atomicOr(&chosen[jj >> 5], 1u << (jj & 31));
-      }
+      rank_cut(cand_rel, cand_j, static_cast<int>(s_ncand), s_remaining, &s_cut_rel, &s_cut_j);
       __syncthreads();
       top = 0;
     } else if (s_mode == 1) {
@@ -529,10 +549,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   // ---- ascending compaction, one contiguous index range per warp
   // mode 0: rel > T, plus the need_eq lowest-index keys with rel == T
   // mode 1: rel >= T (the floor of a bin that is taken whole)
-  // mode 2: rel at or above the floor of the next bin, plus ranked members
+  // mode 2: (rel, index) at or above the cut found by ranking the bin
   const int mode = s_mode;
   const uint32_t T = s_prefix;
-  const uint64_t next_floor = static_cast<uint64_t>(T) + (1ull << shift);
+  const uint32_t cut_rel = s_cut_rel;
+  const int cut_j = s_cut_j;
   const uint32_t need_eq = s_remaining;
   const int nw = blockDim.x >> 5;
   const int chunk = (((Mo + 31) / 32 + nw - 1) / nw) * 32;
@@ -540,7 +561,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   auto plain_take = [&](int j, uint32_t rel) -> bool {
     if (mode == 0) return rel > T;
     if (mode == 1) return rel >= T;
-    return static_cast<uint64_t>(rel) >= next_floor || ((chosen[j >> 5] >> (j & 31)) & 1u);
+    return at_or_above(rel, j, cut_rel, cut_j);
   };
   uint32_t cnt = 0, cnt_eq = 0;
   for (int b0 = wb; b0 < we; b0 += 32) {
@@ -604,12 +625,11 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t cand_rel[kCand];
   __shared__ int cand_j[kCand];
-  __shared__ uint32_t chosen[KPT * 32];           // bitmap over block ids (ranked candidates)
   __shared__ uint32_t tab[KPT * 32];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t red_min[32], red_max[32];
-  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand;
-  __shared__ int s_mode;
+  __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand, s_cut_rel;
+  __shared__ int s_mode, s_cut_j;
   grid_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
@@ -641,7 +661,6 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
     if (tid + k * kSelThreads < Mo) { kmin = min(kmin, kr[k]); kmax = max(kmax, kr[k]); }
   }
   for (int b = tid; b < kBins; b += blockDim.x) hist[b] = 0u;
-  if (tid < KPT * 32) chosen[tid] = 0u;
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if (lane == 0) { red_min[warp] = kmin; red_max[warp] = kmax; }
@@ -698,18 +717,7 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
         }
       }
       __syncthreads();
-      const int c = static_cast<int>(s_ncand);
-      const uint32_t take = s_remaining;
-      for (int i = tid; i < c; i += blockDim.x) {
-        const uint32_t r = cand_rel[i];
-        const int jj = cand_j[i];
-        uint32_t rank = 0;
-        for (int k = 0; k < c; ++k) {
-          const uint32_t rk = cand_rel[k];
-          rank += (rk > r) || (rk == r && cand_j[k] < jj);
-        }
-        if (rank < take) atomicOr(&chosen[jj >> 5], 1u << (jj & 31));
-      }
+      rank_cut(cand_rel, cand_j, static_cast<int>(s_ncand), s_remaining, &s_cut_rel, &s_cut_j);
       __syncthreads();
       top = 0;
     } else if (s_mode == 1) {
@@ -756,21 +764,19 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
     __syncthreads();
     top = s_mode == 1 ? 0 : sh;
   }
+  // kept: mode 0 rel > T plus the need_eq lowest indices with rel == T;
+  // mode 1 rel >= T (the threshold bin whole); mode 2 at or above the cut
   const int mode = s_mode;
   const uint32_t T = s_prefix;
-  const uint64_t next_floor = static_cast<uint64_t>(T) + (1ull << shift);
   const uint32_t need_eq = s_remaining;
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t take = 0u;                              // bit k: block tid + 1024 k is kept
+  {
+    const uint32_t cut_rel = mode == 2 ? s_cut_rel : T;
+    const int cut_j = mode == 1 ? 0x7fffffff : (mode == 2 ? s_cut_j : -1);
 #pragma unroll
-  for (int k = 0; k < KPT; ++k) {
-    const uint32_t rel = kr[k];
-    const int j = tid + k * kSelThreads;
-    bool t;
-    if (mode == 0) t = rel > T;
-    else if (mode == 1) t = rel >= T;
-    else t = static_cast<uint64_t>(rel) >= next_floor || ((chosen[j >> 5] >> (j & 31)) & 1u);
-    if (valid(k) && t) take |= 1u << k;
+    for (int k = 0; k < KPT; ++k)
+      if (valid(k) && at_or_above(kr[k], tid + k * kSelThreads, cut_rel, cut_j)) take |= 1u << k;
   }
   if (mode == 0) {
     // keys equal to the threshold: the need_eq lowest indices
@@ -813,18 +819,14 @@ cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int
   const SelRows rl{lens, len, r, n_min};
   if (M > kSelMaxM) return cudaErrorInvalidValue;
   const bool in_smem = M <= kSelSmemKeys;
-  const size_t bitmap = static_cast<size_t>((M + 31) / 32) * sizeof(uint32_t);
-  const size_t smem = (in_smem ? static_cast<size_t>(M) * sizeof(uint32_t) : 0) + bitmap;
+  const size_t smem = in_smem ? static_cast<size_t>(M) * sizeof(uint32_t) : 0;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const int most = kSelSmemKeys * static_cast<int>(sizeof(uint32_t)) + (kSelMaxM / 32) * 4;
+    const int most = kSelSmemKeys * static_cast<int>(sizeof(uint32_t));
     cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               most);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
