@@ -73,37 +73,56 @@ __device__ __forceinline__ void split_range(const AttnK& a, int s, int64_t len_r
   i1 = static_cast<int>(static_cast<int64_t>(s + 1) * n / a.S);
 }
 
+// Row stride (floats) of the per-warp outputs in shared memory: 4 floats of
+// padding put the rows of heads 2c and 2c + 1 of the tensor-core layout on
+// different banks.
+__host__ __device__ constexpr int merge_row(int D) { return D + 4; }
+// floats of shared memory the per-warp merge needs
+__host__ __device__ constexpr int merge_floats(int D, int NW) { return NW * 8 * merge_row(D) + 2 * NW * 8; }
+
 // Merge the per-warp (m, l, O) of one CTA through shared memory. With one
 // split the CTA writes the normalised output; otherwise it writes its partial
 // and the last CTA of the (row, group) to arrive merges all S partials
 // (log-sum-exp weights) into the output and resets the arrival counter.
-// sm must hold NW * 8 * (D + 2) floats; it is reused by the final merge.
+// sm must hold merge_floats(D, NW) floats; it is reused by the final merge.
 template <typename T, int D, int NW>
 __device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, int g, int s_idx) {
-  float* sm_o = sm;                       // [NW][8][D]
-  float* sm_m = sm + NW * 8 * D;          // [NW][8]
+  constexpr int OR = merge_row(D);
+  float* sm_o = sm;                       // [NW][8][OR]
+  float* sm_m = sm + NW * 8 * OR;         // [NW][8]
   float* sm_l = sm_m + NW * 8;            // [NW][8]
   __shared__ int s_last;
   T* out = static_cast<T*>(a.out);
   const int64_t head0 = static_cast<int64_t>(br) * a.Hq + g * a.G;
-  for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
-    const int h = idx / D, ch = idx % D;
+  constexpr int NT = NW * 32;
+  constexpr int HALF = D / 2;
+  // One output channel pair (c, c + HALF) of one head per thread when the
+  // group fits (G * D / 2 <= threads), so the warp weights are computed once
+  // per pair; otherwise a strided walk over single channels.
+  const bool paired = a.G * HALF <= NT;
+  const int n_items = paired ? a.G * HALF : a.G * D;
+  for (int idx = threadIdx.x; idx < n_items; idx += NT) {
+    const int h = paired ? idx / HALF : idx / D;
+    const int ch = paired ? idx % HALF : idx % D;
     float mstar = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) mstar = fmaxf(mstar, sm_m[w * 8 + h]);
-    float o = 0.f, l = 0.f;
+    float o0 = 0.f, o1 = 0.f, l = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const float sc = mstar == -INFINITY ? 0.f : exp2f(sm_m[w * 8 + h] - mstar);
-      o = fmaf(sc, sm_o[(w * 8 + h) * D + ch], o);
+      o0 = fmaf(sc, sm_o[(w * 8 + h) * OR + ch], o0);
+      if (paired) o1 = fmaf(sc, sm_o[(w * 8 + h) * OR + ch + HALF], o1);
       l = fmaf(sc, sm_l[w * 8 + h], l);
     }
     if (a.S == 1) {
-      out[(head0 + h) * D + ch] = Dt<T>::from_f(o / l);
+      out[(head0 + h) * D + ch] = Dt<T>::from_f(o0 / l);
+      if (paired) out[(head0 + h) * D + ch + HALF] = Dt<T>::from_f(o1 / l);
       if (a.lse != nullptr && ch == 0) a.lse[head0 + h] = (mstar + log2f(l)) * 0.69314718055994531f;
     } else {
       const int64_t row = (head0 + h) * a.S + s_idx;
-      a.part_o[row * D + ch] = o;
+      a.part_o[row * D + ch] = o0;
+      if (paired) a.part_o[row * D + ch + HALF] = o1;
       if (ch == 0) {
         a.part_ml[row * 2] = mstar;
         a.part_ml[row * 2 + 1] = l;
@@ -118,9 +137,8 @@ __device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, in
   if (threadIdx.x == 0) s_last = atomic_add_acq_rel(counter, 1) == a.S - 1;
   __syncthreads();
   if (!s_last) return;
-  // last CTA: each thread merges its (head, channel) outputs over all splits.
-  constexpr int NT = NW * 32;
-  if (a.G * D <= 2 * NT && a.S <= 32) {
+  // last CTA: each thread merges its outputs over all splits.
+  if (paired && a.S <= 32) {
     // common case (at most two outputs per thread, at most 32 splits): every
     // partial output and every (m, l) pair is requested before any is used,
     // so the merge costs one round trip to L2
@@ -173,7 +191,7 @@ __device__ __forceinline__ void cta_finish(const AttnK& a, float* sm, int br, in
   }
   // general case: chunks of up to 32 splits, each loaded in one round trip
   // and folded in with an online log-sum-exp
-  for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
+  for (int idx = threadIdx.x; idx < a.G * D; idx += NT) {
     const int h = idx / D, ch = idx % D;
     const float* po = a.part_o + (head0 + h) * a.S * D + ch;
     const float* ml = a.part_ml + (head0 + h) * a.S * 2;
@@ -425,22 +443,28 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   l1 += __shfl_xor_sync(0xffffffffu, l1, 8);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 16);
 
+  // per-warp partials; head columns past G (padding of the n = 8 product)
+  // are never read and not stored
+  static_assert(merge_floats(D, NW) * 4 <= NW * STAGES * Cfg::kTile, "merge area");
+  constexpr int OR = merge_row(D);
   float* sm = reinterpret_cast<float*>(tiles);
   float* sm_o = sm;
-  float* sm_m = sm + NW * 8 * D;
+  float* sm_m = sm + NW * 8 * OR;
   float* sm_l = sm_m + NW * 8;
   const int h0 = 2 * cq, h1 = 2 * cq + 1;
-  if (gq == 0) {
+  if (gq == 0 && h0 < a.G) {
     sm_m[warp * 8 + h0] = m0; sm_l[warp * 8 + h0] = l0;
     sm_m[warp * 8 + h1] = m1; sm_l[warp * 8 + h1] = l1;
   }
+  if (h0 < a.G) {
 #pragma unroll
-  for (int mt = 0; mt < KT; ++mt) {
-    const int ch = mt * 16 + gq;
-    sm_o[(warp * 8 + h0) * D + ch] = o[mt][0];
-    sm_o[(warp * 8 + h1) * D + ch] = o[mt][1];
-    sm_o[(warp * 8 + h0) * D + ch + 8] = o[mt][2];
-    sm_o[(warp * 8 + h1) * D + ch + 8] = o[mt][3];
+    for (int mt = 0; mt < KT; ++mt) {
+      const int ch = mt * 16 + gq;
+      sm_o[(warp * 8 + h0) * OR + ch] = o[mt][0];
+      sm_o[(warp * 8 + h1) * OR + ch] = o[mt][1];
+      sm_o[(warp * 8 + h0) * OR + ch + 8] = o[mt][2];
+      sm_o[(warp * 8 + h1) * OR + ch + 8] = o[mt][3];
+    }
   }
   __syncthreads();
   cta_finish<__nv_bfloat16, D, NW>(a, sm, br, g, s_idx);
@@ -542,16 +566,17 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
     }
   }
   __syncthreads();
-  float* sm = tiles;                       // reuse: needs NW*8*(D+2) floats
+  float* sm = tiles;                       // reuse: needs merge_floats(D, NW) floats
+  constexpr int OR = merge_row(D);
   float* sm_o = sm;
-  float* sm_m = sm + NW * 8 * D;
+  float* sm_m = sm + NW * 8 * OR;
   float* sm_l = sm_m + NW * 8;
 #pragma unroll
   for (int h = 0; h < 8; ++h) {
     if (h < a.G) {
       if (lane == 0) { sm_m[warp * 8 + h] = m[h]; sm_l[warp * 8 + h] = l[h]; }
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) sm_o[(warp * 8 + h) * D + lane + 32 * i] = acc[h][i];
+      for (int i = 0; i < CPL; ++i) sm_o[(warp * 8 + h) * OR + lane + 32 * i] = acc[h][i];
     }
   }
   __syncthreads();
@@ -592,7 +617,7 @@ template <int D>
 static cudaError_t attend_f32_t(const Shape& s, const AttnK& k, const AttnArgs& a,
                                 cudaStream_t st) {
   const size_t tiles = static_cast<size_t>(kNW) * 2 * 16 * (D + 1);
-  const size_t merge = static_cast<size_t>(kNW) * 8 * (D + 2);
+  const size_t merge = static_cast<size_t>(merge_floats(D, kNW));
   const size_t smem = (8 * D + (tiles > merge ? tiles : merge)) * sizeof(float);
   static bool attr_set[64] = {false};
   int dev = 0;

@@ -156,6 +156,34 @@ def test_crowded_ties_take_lowest_indices():
         assert np.array_equal(res["gpu_sel"], res["sel"])
 
 
+@pytest.mark.parametrize("extra", [0, 5, 700, 1500])
+def test_two_score_levels(extra):
+    """Blocks whose tokens alternate +a and -a in every channel have lo = -a,
+    hi = +a and the pooled bound a * sum_c (P_c - N_c) >= 0, so two amplitudes
+    give exactly two scores. With need + extra blocks at the higher one the
+    threshold bin is taken whole (0), resolved by ranking its members by index
+    (5, 700) or, with more members than the ranked path holds, by the radix
+    passes (1500). Either way the lowest-index high blocks are kept."""
+    spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=16 * 3000, steps=1,
+                dtype="bf16", r=0.1, n_min=4)
+    K, V = make_cache(spec)
+    M = orc.num_blocks(spec.len0 + 1)
+    need = orc.num_selected(M, spec.r, spec.n_min) - 1
+    rng = np.random.default_rng(7)
+    amp = np.full((2, 3000), 0.5, dtype=np.float32)
+    for h in range(2):
+        amp[h, rng.choice(3000, need + extra, replace=False)] = 1.0
+    sign = np.where(np.arange(16) % 2 == 0, 1.0, -1.0).astype(np.float32)
+    blocks = amp[:, :, None, None] * sign[None, None, :, None] * np.ones(128, np.float32)
+    K[0, :, :spec.len0] = blocks.reshape(2, spec.len0, 128)
+    p = Pair(spec, cache=(K, V))
+    res = p.decode(0)
+    for h in range(2):
+        high = np.sort(np.nonzero(amp[h] == 1.0)[0])[:need]
+        assert list(res["gpu_sel"][0, h]) == list(high) + [M - 1]
+    assert np.array_equal(res["gpu_sel"], res["sel"])
+
+
 @pytest.mark.parametrize("len0", [16 * 2000 + 5, 16 * 6000, 16 * 12000 + 3, 16 * 30000])
 def test_select_row_sizes(len0):
     """Rows of 2000 to 30000 blocks: the register selection with 8 and 16 keys
