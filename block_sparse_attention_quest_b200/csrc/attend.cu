@@ -268,9 +268,6 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
 
-  // the next kernel in the stream may start its prologue now (whatever it
-  // reads from this kernel it reads after its own dependency wait)
-  grid_launch_dependents();
   const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
   const int b = br / a.R, r = br % a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -427,6 +424,11 @@ __global__ void __launch_bounds__(NW * 32) attend_bf16_kernel(const __grid_const
       issue(k + STAGES);
     }
   }
+  // The next kernel in the stream may launch once every CTA has streamed its
+  // blocks (whatever it reads from this kernel it reads after its own
+  // dependency wait); launched earlier its prologue would compete with the
+  // stream, launched here it overlaps the merge tail.
+  grid_launch_dependents();
   if (!ok) {
     // drain the copies this warp still has in flight (bounded), then leave
     // without writing a partial; the host sees the error flag
@@ -478,7 +480,6 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
   extern __shared__ float smf[];
   float* sq = smf;                            // [8][D]
   float* tiles = smf + 8 * D;                 // [NW][2][16][P]
-  grid_launch_dependents();
   const int s_idx = blockIdx.x, g = blockIdx.y, br = blockIdx.z;
   const int b = br / a.R, r = br % a.R;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -565,6 +566,7 @@ __global__ void __launch_bounds__(NW * 32) attend_f32_kernel(AttnK a) {
       }
     }
   }
+  grid_launch_dependents();                   // see the bf16 kernel
   __syncthreads();
   float* sm = tiles;                       // reuse: needs merge_floats(D, NW) floats
   constexpr int OR = merge_row(D);

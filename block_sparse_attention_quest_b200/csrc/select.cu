@@ -94,21 +94,31 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   constexpr int NW = 8;
 
   __shared__ float coef[2 * D];                    // [N (for lo) | P (for hi)]
-  // launched as a programmatic dependent of whatever precedes it in the
-  // stream (q, the cache and the descriptors may come from there): nothing is
-  // read before the wait, only the launch overlaps the previous kernel's tail
-  grid_dependency_wait();
-  grid_launch_dependents();
   const int g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(b) * a.H + g;
+  const T* dbase = static_cast<const T*>(a.desc) + bh * a.Mmax * 2 * D;
+  // Launched as a programmatic dependent of whatever precedes it in the
+  // stream (q, the cache and the descriptors may come from there): nothing is
+  // read before the wait. This CTA's descriptor chunk (for the length bound)
+  // is only prefetched into L2, which overlaps its HBM fetch with the
+  // previous kernel's tail; the loads after the wait see that kernel's writes.
+  {
+    const int jb = blockIdx.x * a.blocks_per_cta;
+    const int je = min(jb + a.blocks_per_cta, a.M - 1);
+    const char* c0 = reinterpret_cast<const char*>(dbase + static_cast<int64_t>(jb) * 2 * D);
+    const int64_t bytes = static_cast<int64_t>(max(je - jb, 0)) * 2 * D * sizeof(T);
+    for (int64_t off = static_cast<int64_t>(tid) * 128; off < bytes; off += 256 * 128)
+      prefetch_l2(c0 + off);
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int64_t len_b = row_len(a.lens, a.len, b);
   if (a.lens != nullptr && blockIdx.x == 0 && g == 0 && tid == 0 && row_len_bad(a.lens, a.len, b))
     raise_error(a.ctrl, kErrBadIndex);
   const int last_scored = static_cast<int>((len_b + kBlock - 1) / kBlock) - 1;  // block M-1 is forced, not scored
   const int j_begin = blockIdx.x * a.blocks_per_cta;
   const int j_end = min(j_begin + a.blocks_per_cta, last_scored);
-  const T* dbase = static_cast<const T*>(a.desc) + bh * a.Mmax * 2 * D;
   float* sout = a.scores + bh * a.M;
   const int seg = lane / W;
 
