@@ -44,7 +44,7 @@ METRIC = "ReSA decode-step us & achieved HBM GB/s vs roofline at 128K/256K; rect
 # DRAM bytes (read + write) per launch of the attention kernel from one ncu
 # capture of this workload (profiles/attend_bf16_kernel_128k.md). Reset an
 # entry to None whenever attend_bf16_kernel changes.
-NCU_TRAFFIC = {"resa_decode_128k_b1": 54238976}
+NCU_TRAFFIC = {"resa_decode_128k_b1": 53982720}
 
 
 def parse():
