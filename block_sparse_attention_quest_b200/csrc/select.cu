@@ -100,14 +100,18 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
   const T* dbase = static_cast<const T*>(a.desc) + bh * a.Mmax * 2 * D;
   // Launched as a programmatic dependent of whatever precedes it in the
   // stream (q, the cache and the descriptors may come from there): nothing is
-  // read before the wait. This CTA's descriptor chunk (for the length bound)
-  // is only prefetched into L2, which overlaps its HBM fetch with the
-  // previous kernel's tail; the loads after the wait see that kernel's writes.
+  // read before the wait. The start of this CTA's descriptor chunk (for the
+  // length bound) is only prefetched into L2, which overlaps its HBM fetch with
+  // the previous kernel's tail; the loads after the wait see that kernel's
+  // writes. At most kPrefetchBytes per CTA: a larger prefetch delays the
+  // previous kernel's own tail (its merge round trips queue behind it).
   {
+    constexpr int64_t kPrefetchBytes = 80 * 1024;
     const int jb = blockIdx.x * a.blocks_per_cta;
     const int je = min(jb + a.blocks_per_cta, a.M - 1);
     const char* c0 = reinterpret_cast<const char*>(dbase + static_cast<int64_t>(jb) * 2 * D);
-    const int64_t bytes = static_cast<int64_t>(max(je - jb, 0)) * 2 * D * sizeof(T);
+    const int64_t bytes = min(static_cast<int64_t>(max(je - jb, 0)) * 2 * D * sizeof(T),
+                              kPrefetchBytes);
     for (int64_t off = static_cast<int64_t>(tid) * 128; off < bytes; off += 256 * 128)
       prefetch_l2(c0 + off);
   }
