@@ -593,7 +593,7 @@ template <int D>
 static cudaError_t attend_bf16_t(const Shape& s, const AttnK& k, const AttnArgs& a,
                                  cudaStream_t st) {
   using Cfg = Bf16Cfg<D, kNW, kStages>;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; launches may come from several host threads
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
@@ -621,7 +621,7 @@ static cudaError_t attend_f32_t(const Shape& s, const AttnK& k, const AttnArgs& 
   const size_t tiles = static_cast<size_t>(kNW) * 2 * 16 * (D + 1);
   const size_t merge = static_cast<size_t>(merge_floats(D, kNW));
   const size_t smem = (8 * D + (tiles > merge ? tiles : merge)) * sizeof(float);
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; launches may come from several host threads
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {

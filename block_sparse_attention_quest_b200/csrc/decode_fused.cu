@@ -699,7 +699,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(const __grid
 template <int D>
 static cudaError_t fused_t(const FusedLaunch& f, cudaStream_t st) {
   using Cfg = FCfg<D>;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; launches may come from several host threads
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;

@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const float* __restrict
 template <int D>
 static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   using C = RectCfg<D>;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; launches may come from several host threads
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;

@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
 template <typename T, int D>
 static cudaError_t score_t(const Shape& s, const ScoreArgs& a0, int num_sms, cudaStream_t st) {
   ScoreArgs a = a0;
-  static int occ[64] = {0};
+  static std::atomic<int> occ[64];         // per device; launches may come from several host threads
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -834,7 +834,7 @@ cudaError_t launch_select(const Shape& s, const float* scores, int32_t* sel, int
   if (M > kSelMaxM) return cudaErrorInvalidValue;
   const bool in_smem = M <= kSelSmemKeys;
   const size_t smem = in_smem ? static_cast<size_t>(M) * sizeof(uint32_t) : 0;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];   // per device; launches may come from several host threads
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
