@@ -413,6 +413,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
   __shared__ int s_mode;                          // 0 exact threshold, 1 bin floor, 2 ranked bin
   __shared__ int s_cut_j;
   grid_launch_dependents();
+  // Scores come from the previous kernel. The wait comes before every exit,
+  // the early ones included: the attention kernel launched after this one
+  // waits only for this grid, so this wait is also what orders it after the
+  // score kernel's append of the new token (block M-1 is always attended).
+  grid_dependency_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
   const float* s = scores + bh * M;
@@ -430,7 +435,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const float* __rest
     if (tid == 0) out[0] = M - 1;
     return;
   }
-  grid_dependency_wait();                          // scores come from the previous kernel
   auto key_at = [&](int j) -> uint32_t {
     if constexpr (IN_SMEM) return skeys[j];
     else return score_key(__ldcg(s + j));
@@ -645,6 +649,7 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
   __shared__ uint32_t s_prefix, s_remaining, s_total, s_kmin, s_kmax, s_ncand, s_cut_rel;
   __shared__ int s_mode, s_cut_j;
   grid_launch_dependents();
+  grid_dependency_wait();                          // before every exit (see select_kernel)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.y) * H + blockIdx.x;
   const float* s = scores + bh * M;
@@ -660,7 +665,6 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const float* __
     if (tid == 0) out[0] = M - 1;
     return;
   }
-  grid_dependency_wait();                          // scores come from the previous kernel
   uint32_t kr[KPT];
   float x[KPT];
 #pragma unroll
