@@ -42,7 +42,7 @@ EXPORTED = ("resa_num_selected", "resa_workspace_bytes", "resa_build_desc",
             "resa_decode_dense", "resa_rectify",
             "resa_workspace_status", "resa_status_string", "resa_decode_sparse_noalloc",
             "resa_build_desc_varlen", "resa_decode_sparse_varlen", "resa_decode_dense_varlen",
-            "resa_rectify_varlen", "resa_prefill", "resa_wait_check")
+            "resa_rectify_varlen", "resa_prefill", "resa_wait_check", "resa_noalloc_status")
 
 
 class Dims(ctypes.Structure):
@@ -100,6 +100,8 @@ _lib.resa_wait_check.restype = ctypes.c_int
 _lib.resa_wait_check.argtypes = [_P, ctypes.c_int32, ctypes.c_uint32, _P, _P]
 _lib.resa_workspace_status.restype = ctypes.c_int
 _lib.resa_workspace_status.argtypes = [_P, _P]
+_lib.resa_noalloc_status.restype = ctypes.c_int
+_lib.resa_noalloc_status.argtypes = [_P]
 _lib.resa_status_string.restype = ctypes.c_char_p
 _lib.resa_status_string.argtypes = [ctypes.c_int]
 
@@ -226,6 +228,12 @@ def decode_sparse_noalloc(q, k_new, v_new, k_cache, v_cache, desc, length: int, 
         ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
         _ptr(desc), int(length), float(r), int(n_min), float(softmax_scale), _ptr(out), _ptr(lse),
         _ptr(sel), _stream(stream)), "resa_decode_sparse_noalloc")
+
+
+def noalloc_status(stream=None) -> int:
+    """Synchronise and read (and clear) the device error flag of the fixed
+    scratch that decode_sparse_noalloc uses on the current device."""
+    return _lib.resa_noalloc_status(_stream(stream))
 
 
 def workspace_status(workspace, stream=None) -> int:

@@ -13,7 +13,13 @@
 // that loads libresa.so holds it until the process exits. In host code its
 // name only stands in for the symbol, so the device address is looked up with
 // cudaGetSymbolAddress once per device (on that device's first call) and
-// cached.
+// cached. A failed call drops the cached address, so a context rebuilt after
+// cudaDeviceReset looks it up again.
+//
+// The array's first 256 bytes are the same control block a caller workspace
+// starts with: its error word is sticky across calls (a timed-out wait or a
+// bad block id raised by one call stays set until resa_noalloc_status reads
+// and clears it); the arrival counters after it are cleared by every call.
 #include <mutex>
 
 #include "../../include/resa.h"
@@ -42,6 +48,14 @@ void* scratch_address() {
   return g_addr[dev];
 }
 
+// forget the current device's cached address (after a CUDA failure)
+void drop_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_addr[dev] = nullptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -64,11 +78,27 @@ int resa_decode_sparse_noalloc(const resa_dims* dims, const void* q, const void*
   s.bf16 = dims->dtype == RESA_BF16;
   void* ws = scratch_address();
   if (ws == nullptr) return RESA_ERR_CUDA;
-  // the error word and the arrival counters must start at zero
+  // the arrival counters must start at zero; the error word (the first bytes
+  // of the control block) is left for resa_noalloc_status to read
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, resa::workspace_zero_prefix(s), st) != cudaSuccess) return RESA_ERR_CUDA;
-  return resa_decode_sparse(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min,
-                            softmax_scale, out, lse, sel, ws, kScratchBytes, stream);
+  const size_t zero_end = resa::workspace_zero_prefix(s);
+  if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + resa::kCtrlBytes, 0,
+                      zero_end - resa::kCtrlBytes, st) != cudaSuccess) {
+    drop_scratch_address();
+    return RESA_ERR_CUDA;
+  }
+  const int rc = resa_decode_sparse(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min,
+                                    softmax_scale, out, lse, sel, ws, kScratchBytes, stream);
+  if (rc == RESA_ERR_CUDA) drop_scratch_address();
+  return rc;
+}
+
+int resa_noalloc_status(void* stream) {
+  void* ws = scratch_address();
+  if (ws == nullptr) return RESA_ERR_CUDA;
+  const int rc = resa_workspace_status(ws, stream);
+  if (rc == RESA_ERR_CUDA) drop_scratch_address();
+  return rc;
 }
 
 }  // extern "C"

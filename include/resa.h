@@ -187,17 +187,29 @@ RESA_API int resa_rectify(const resa_dims* dims, const void* q_f, const void* k_
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) and caches it; make that first call outside any
  *    stream capture.
- *  - Each call clears the array's error word and counters on `stream`
+ *  - Each call clears the array's arrival counters on `stream`
  *    (cudaMemsetAsync), then runs resa_decode_sparse on it. It allocates
  *    nothing. All calls on a device share the one array: calls that may
  *    overlap on the GPU (different streams, different threads) race and must
  *    be serialised by the caller.
+ *  - Device-side errors (a timed-out wait, a bad block id) set the array's
+ *    error word, which stays set across later calls until
+ *    resa_noalloc_status() reads and clears it.
+ *  - After cudaDeviceReset the first call must again come outside any
+ *    stream capture (a failed call forgets the cached address).
  * Arguments and results are those of resa_decode_sparse. */
 RESA_API int resa_decode_sparse_noalloc(const resa_dims* dims, const void* q, const void* k_new,
                                         const void* v_new, void* k_cache, void* v_cache,
                                         void* desc, int64_t len, double r, int32_t n_min,
                                         float softmax_scale, void* out, float* lse,
                                         int32_t* sel, void* stream);
+
+/* Device error flags of the array resa_decode_sparse_noalloc uses on the
+ * current device (no counterpart in the method): synchronises `stream`, then
+ * reads and clears them, as resa_workspace_status() does for a caller
+ * workspace. Returns RESA_OK, RESA_ERR_TIMEOUT, RESA_ERR_BAD_INDEX or
+ * RESA_ERR_CUDA. */
+RESA_API int resa_noalloc_status(void* stream);
 
 /* Prefill-side step: dense causal attention of every position of a prompt,
  * with the Quest descriptors of its keys produced by the same pass ("Rectified

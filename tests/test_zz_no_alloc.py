@@ -1,10 +1,15 @@
-"""The allocation-free decode entry point against the workspace one.
+"""The allocation-free decode entry point, against the oracle and against the
+workspace entry point.
 
-resa_decode_sparse_noalloc serves callers that cannot allocate device memory
-(a framework allocator owns the GPU, a graph-captured decode loop, a plugin
-host that passes only tensors). It keeps its scratch in a fixed array inside
-the library. This file is collected last so that a failure here never hides
-the other GPU tests; it also runs on its own in a fresh process.
+Some callers cannot allocate device memory: code inside a framework whose
+caching allocator owns the GPU (a private cudaMalloc there can fail once the
+pool has reserved the memory, and bypasses its accounting), decode loops
+captured into CUDA graphs that must not allocate between captures, and plugin
+hosts that hand a kernel only its input and output pointers.
+resa_decode_sparse_noalloc serves them with scratch in a fixed array inside
+the library, and resa_noalloc_status reports the device-side errors raised
+there. This file is collected last so that a failure here never hides the
+other GPU tests; it also runs on its own in a fresh process.
 """
 import ctypes
 
@@ -12,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as orc
 from workload import Spec, decode_inputs, make_cache
 
 pytestmark = pytest.mark.gpu
@@ -20,20 +26,22 @@ TOL = (5e-3, 2e-2)   # bf16: rel-L2, max-abs (the tolerance of the parity tests)
 
 
 def _close(a, b):
-    a = a.float().cpu().numpy().astype(np.float64)
-    b = b.float().cpu().numpy().astype(np.float64)
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
     rel = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
     assert rel <= TOL[0] and np.abs(a - b).max() <= TOL[1], rel
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+def test_noalloc_matches_oracle_and_workspace_entry_point_on_two_calls():
     import __graft_entry__
     __graft_entry__.build()
     import block_sparse_attention_quest_b200 as resa
+    from tests.pair import check_selection, fp32_score_error
 
     spec = Spec(batch=2, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=5000, steps=2,
                 dtype="bf16", r=0.1, n_min=16)
     K, V = make_cache(spec)
+    st = orc.State(K, V, spec.len0, spec.group)
 
     def dev(x):
         return torch.from_numpy(np.ascontiguousarray(x)).cuda().to(torch.bfloat16)
@@ -50,7 +58,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     stream = torch.cuda.current_stream().cuda_stream
     for step in range(2):                       # two calls in a row
         length = spec.len0 + step + 1
-        q, kn, vn = (dev(x) for x in decode_inputs(spec, step))
+        q_h, kn_h, vn_h = decode_inputs(spec, step)
+        q, kn, vn = dev(q_h), dev(kn_h), dev(vn_h)
         n = resa.num_selected(length, spec.r, spec.n_min)
         out_a = torch.empty(2, 32, 128, dtype=torch.bfloat16, device="cuda")
         out_b = torch.empty_like(out_a)
@@ -65,8 +74,19 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
             vb.data_ptr(), db.data_ptr(), length, spec.r, spec.n_min, 1.0, out_b.data_ptr(),
             lse_b.data_ptr(), sel_b.data_ptr(), stream)
         assert rc == resa.RESA_OK, resa.status_string(rc)
-        torch.cuda.synchronize()
-        _close(out_b, out_a)
+        assert resa._lib.resa_noalloc_status(stream) == resa.RESA_OK
+        assert resa.workspace_status(ws) == resa.RESA_OK
+        # against the oracle (selection by the parity rule, outputs within tolerance)
+        ref = st.decode(q_h, kn_h, vn_h, spec.r, spec.n_min, 1.0)
+        gsel = sel_b.cpu().numpy()
+        err = fp32_score_error(q_h, st.lo, st.hi, ref["scores"].shape[-1])
+        exact = all(check_selection(gsel[b, g], ref["scores"][b, g], n, err[b, g])
+                    for b in range(2) for g in range(8))
+        O, L = (ref["out"], ref["lse"]) if exact else st.attend_with(q_h, gsel, 1.0)
+        _close(out_b.float().cpu().numpy(), O)
+        _close(lse_b.cpu().numpy(), L)
+        # against the workspace entry point on the same inputs
+        _close(out_b.float().cpu().numpy(), out_a.float().cpu().numpy())
         assert torch.allclose(lse_b, lse_a, rtol=0, atol=1e-4)
         assert torch.equal(sel_b, sel_a)
         assert torch.equal(kb, ka) and torch.equal(vb, va) and torch.equal(db, da)
