@@ -37,10 +37,51 @@ def close(got, ref, dtype: str, what: str = ""):
     return rel, mx
 
 
-def check_selection(gpu_sel: np.ndarray, scores: np.ndarray, n: int):
-    """Gap rule on one (b, g). Returns True when the GPU set must equal the
-    oracle's (and does); False when near-tied (the GPU choice is then only
-    checked for validity)."""
+# (step, KV group) decisions seen by check_selection: "exact" ones were
+# asserted equal to the oracle's set, "near_tie" ones passed the band checks
+SELECTION_STATS = {"exact": 0, "near_tie": 0}
+
+
+def fp32_score_error(q: np.ndarray, lo: np.ndarray, hi: np.ndarray, M: int) -> np.ndarray:
+    """Bound on |fp32 score - exact score| for every block of every group.
+
+    The kernel folds the group into N_c = sum_h min(q_hc, 0) and
+    P_c = sum_h max(q_hc, 0) (G fp32 additions) and sums the 2d products
+    N_c lo_c and P_c hi_c in some fp32 order; whatever the order, the error
+    of such a sum is at most gamma_k times the sum of the products' magnitudes
+    (gamma_k = k u / (1 - k u), u = 2^-24, k >= number of rounded operations
+    on any path), and that sum is at most sum_c (sum_h |q_hc|) max(|lo_c|, |hi_c|).
+    q: [B, Hq, d]; lo, hi: [B, Hkv, >= M, d]. Returns [B, Hkv, M]."""
+    B, Hq, d = q.shape
+    H = lo.shape[1]
+    G = Hq // H
+    k = 2 * d + G + 2
+    u = 2.0 ** -24
+    gamma = k * u / (1.0 - k * u)
+    qa = np.abs(np.asarray(q, np.float64)).reshape(B, H, G, d).sum(axis=2)       # [B, H, d]
+    mx = np.maximum(np.abs(np.asarray(lo[:, :, :M], np.float64)),
+                    np.abs(np.asarray(hi[:, :, :M], np.float64)))                # [B, H, M, d]
+    return gamma * np.einsum("bhmd,bhd->bhm", mx, qa)
+
+
+def check_selection(gpu_sel: np.ndarray, scores: np.ndarray, n: int,
+                    err: np.ndarray | None = None) -> bool:
+    """Selection parity on one (batch, KV group).
+
+    s_(n) and s_(n+1) are the oracle's (n-1)-th and n-th best scores among the
+    non-local blocks (the local block takes one of the n places). Where their
+    relative gap exceeds GAP the GPU set must equal the oracle's bit-exactly.
+    Otherwise (a near tie, where fp32 and fp64 scores may order blocks
+    differently) with the band B = [s_(n+1) - d, s_(n) + d], d = GAP |s_(n)|:
+      * every non-local block scoring above B is selected;
+      * every other selected block scores inside B (so the list holds exactly
+        n - 1 - #above of them);
+      * no unselected block beats a selected one by more than d.
+    With `err` (a bound on each block's fp32 score error, fp32_score_error),
+    a near tie whose oracle set is separated from the rest by more than the
+    error bounds (min over kept of s - err > max over the others of s + err)
+    cannot be reordered by fp32 rounding, so it must be exact as well.
+    Returns True for an exact decision, False for a near tie."""
     M = scores.shape[0]
     sel = [int(x) for x in gpu_sel]
     assert len(sel) == n, (len(sel), n)
@@ -49,16 +90,35 @@ def check_selection(gpu_sel: np.ndarray, scores: np.ndarray, n: int):
     oracle_sel = [int(x) for x in orc.select_blocks(scores, n)]
     if n == 1 or n >= M:
         assert sel == oracle_sel
+        SELECTION_STATS["exact"] += 1
         return True
-    others = scores[: M - 1]
+    others = np.asarray(scores[: M - 1], dtype=np.float64)
     order = np.lexsort((np.arange(M - 1), -others))
     s_n, s_next = others[order[n - 2]], others[order[n - 1]]
-    scale = max(abs(s_n), 1e-30)
-    if (s_n - s_next) / scale > GAP:
+    d = GAP * max(abs(s_n), 1e-30)
+    if (s_n - s_next) > d:
         assert sel == oracle_sel, "selection differs although the score gap is clear"
+        SELECTION_STATS["exact"] += 1
         return True
-    thr = s_next - GAP * scale
-    assert all(others[j] >= thr for j in sel[:-1]), "selected a block below the near-tie band"
+    if err is not None:
+        e = np.asarray(err[: M - 1], dtype=np.float64)
+        kept, rest_o = order[: n - 1], order[n - 1:]
+        if (others[kept] - e[kept]).min() > (others[rest_o] + e[rest_o]).max():
+            assert sel == oracle_sel, "selection differs although fp32 error cannot reorder it"
+            SELECTION_STATS["exact"] += 1
+            return True
+    chosen = np.asarray(sel[:-1], dtype=np.int64)
+    picked = np.zeros(M - 1, dtype=bool)
+    picked[chosen] = True
+    above = others > s_n + d
+    assert np.all(picked[above]), "a block scoring above the near-tie band was dropped"
+    rest = others[picked & ~above]
+    assert np.all(rest >= s_next - d), "selected a block below the near-tie band"
+    assert rest.size == (n - 1) - int(above.sum())
+    if np.any(~picked):
+        assert others[picked].min() >= others[~picked].max() - d, \
+            "an unselected block beats a selected one by more than the band"
+    SELECTION_STATS["near_tie"] += 1
     return False
 
 
@@ -122,10 +182,13 @@ class Pair:
         else:
             res = self.st.decode(q, kn, vn, self.r, self.n_min, scale)
             gsel = sel[R].cpu().numpy()
+            M = res["scores"].shape[-1]
+            err = fp32_score_error(q, self.st.lo, self.st.hi, M)
             exact = True
             for b in range(len(R)):
                 for g in range(spec.n_kv_heads):
-                    exact &= check_selection(gsel[b, g], res["scores"][b, g], res["n"])
+                    exact &= check_selection(gsel[b, g], res["scores"][b, g], res["n"],
+                                             err[b, g])
             if not exact:   # near-tie somewhere: compare on the GPU's selection
                 O, L = self.st.attend_with(q, gsel, scale)
                 res = dict(res, out=O, lse=L)
