@@ -41,10 +41,40 @@ WORKLOAD_NAMES = {
 }
 METRIC = "ReSA decode-step us & achieved HBM GB/s vs roofline at 128K/256K; rectify us"
 
-# DRAM bytes (read + write) per launch of the attention kernel from one ncu
-# capture of this workload (profiles/attend_bf16_kernel_128k.md). Reset an
-# entry to None whenever attend_bf16_kernel changes.
-NCU_TRAFFIC = {"resa_decode_128k_b1": 53982720}
+# Counters taken from ncu captures of the kernels as they stand, each keyed by
+# a hash of the kernel's source files at capture time: a counter is reported
+# only while the sources still hash to that value (null once a kernel changes).
+#   attention: DRAM read + write bytes per launch of attend_bf16_kernel at the
+#     128K workload (--metrics dram__bytes_read.sum,dram__bytes_write.sum);
+#   rectify: sm__pipe_tensor_cycles_active (% of peak, active cycles) of
+#     rectify_tc_kernel at 128K, f = 32 (--set full, one cold launch).
+NCU_COUNTERS = {
+    "attention": {"files": ["attend.cu", "common.cuh", "launch.h"], "source": None,
+                  "traffic": {"resa_decode_128k_b1": None}},
+    "rectify": {"files": ["rectify_tc.cu", "tc.cuh", "common.cuh", "launch.h"], "source": None,
+                "tensor_pipe_active_pct": None, "traffic": None},
+}
+
+
+def source_hash(files) -> str:
+    """First 16 hex digits of the SHA-256 of the given kernel sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, "block_sparse_attention_quest_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def counter(kind: str, key: str, workload: str | None = None):
+    """A captured counter, or None when the kernel changed since its capture."""
+    c = NCU_COUNTERS[kind]
+    if c["source"] is None or source_hash(c["files"]) != c["source"]:
+        return None
+    v = c.get(key)
+    if isinstance(v, dict):
+        v = v.get(workload)
+    return v
 
 
 def parse():
@@ -60,6 +90,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas (weak scaling) or one layer's KV heads "
+                         "split over the ranks (strong scaling)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the 256K, 32K x 4 and 64K x 16 workloads of the default run")
     return ap.parse_args()
 
 
@@ -133,23 +168,47 @@ def max_over_ranks(value: float, dist, device) -> float:
 
 
 # ----------------------------------------------------------------- GPU arm
-def run_ours(args, rank, world, local_rank):
+def device_cache(spec, dev, tdt):
+    """K, V [B, Hkv, max_len, d] drawn on the device with the workload recipe
+    (N(0, 1) per element plus a N(0, 0.5^2) mean vector per (batch, KV head,
+    block), needles shifted by shift * q_dir), rounded to the cache dtype.
+    Used for the extra benchmark workloads, whose sizes make the host
+    generator slow; the bits differ from the host generator's, the
+    distribution does not."""
     import torch
-    import __graft_entry__
-    __graft_entry__.build()
-    import block_sparse_attention_quest_b200 as resa
-    from workload import config, decode_inputs, make_cache, rectify_inputs
+    from workload import needle_layout
+    B, H, L, d = spec.batch, spec.n_kv_heads, spec.max_len, spec.head_dim
+    g = torch.Generator(device=dev).manual_seed(spec.seed)
+    nb = (spec.len0 + 15) // 16
+    out = []
+    for _ in ("k", "v"):
+        arr = torch.zeros(B, H, L, d, dtype=tdt, device=dev)
+        for b in range(B):
+            mean = 0.5 * torch.randn(H, nb, 1, d, generator=g, device=dev)
+            x = torch.randn(H, nb, 16, d, generator=g, device=dev) + mean
+            arr[b, :, :spec.len0] = x.view(H, nb * 16, d)[:, :spec.len0].to(tdt)
+            del x, mean
+        out.append(arr)
+    if spec.needles:
+        qd, pos = needle_layout(spec)
+        qd_t = torch.from_numpy(qd).to(dev)
+        for b in range(B):
+            for h in range(H):
+                for j in pos[b, h]:
+                    sl = out[0][b, h, int(j) * 16:(int(j) + 1) * 16]
+                    sl.copy_((sl.float() + spec.needle_shift * qd_t[b, h]).to(tdt))
+    return out
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    cfg_idx = WORKLOADS[args.workload]
-    over = {"steps": 64}
-    if args.r is not None:
-        over["r"] = args.r
-    if args.f is not None:
-        over["f"] = args.f
-    spec = config(cfg_idx, **over)
-    f, L = spec.f, args.layers
+
+def measure_workload(args, resa, spec, L, dev, stream, host_cache=True, full=True):
+    """Time one workload: a step of f sparse decode positions on L layer caches
+    plus L rectifications, as a CUDA graph; per-call decode and rectify
+    times; the sparse and dense (r = 1) calls back to back; the attention
+    kernel alone. With full=True also the staged split and the end-to-end
+    run through the Python API with host buffers."""
+    import torch
+    from workload import decode_inputs, make_cache, rectify_inputs
+    f = spec.f
     tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
     esize = 2 if spec.dtype == "bf16" else 4
     B, Hq, H, d = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
@@ -157,9 +216,12 @@ def run_ours(args, rank, world, local_rank):
     def dev_t(x):
         return torch.from_numpy(np.ascontiguousarray(x)).to(dev).to(tdt)
 
-    K, V = make_cache(spec)
-    k0, v0 = dev_t(K), dev_t(V)
-    del K, V
+    if host_cache:
+        K, V = make_cache(spec)
+        k0, v0 = dev_t(K), dev_t(V)
+        del K, V
+    else:
+        k0, v0 = device_cache(spec, dev, tdt)
     layers = []
     for li in range(L):
         k = k0 if li == 0 else k0.clone()
@@ -230,13 +292,13 @@ def run_ours(args, rank, world, local_rank):
             if timing is not None:
                 timing["rect"][li][1].record()
 
-    stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     # eager run once (also validates arguments), then capture
     with torch.cuda.stream(stream):
         step()
     torch.cuda.synchronize()
-    assert resa.workspace_status(ws[0]) == resa.RESA_OK
+    for w in ws:
+        assert resa.workspace_status(w) == resa.RESA_OK
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         step()
@@ -246,72 +308,73 @@ def run_ours(args, rank, world, local_rank):
     graph_t = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_t, stream=stream):
         step(timing)
-    # the same step through the two stage calls (score + select, then
-    # attention): the per-stage split and the attention kernel on its own
-    timing_s = {"dec": [[(mk(), mk(), mk()) for _ in range(L)] for _ in range(f)],
-                "rect": [(mk(), mk()) for _ in range(L)]}
-    graph_s = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_s, stream=stream):
-        step(timing_s, stages=True)
+    graph_s = timing_s = None
+    if full:
+        # the same step through the two stage calls (score + select, then
+        # attention): the per-stage split
+        timing_s = {"dec": [[(mk(), mk(), mk()) for _ in range(L)] for _ in range(f)],
+                    "rect": [(mk(), mk()) for _ in range(L)]}
+        graph_s = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_s, stream=stream):
+            step(timing_s, stages=True)
 
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
+    res = {"graph": graph, "layers": layers, "ws": ws, "dec_in": dec_in, "rect_in": rect_in,
+           "len_start": len_start, "build_desc_us": build_desc_us}
 
-    def barrier():
+    def timed_region(steps, warmup, dist=None, sampler=None):
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        if sampler is not None:
+            sampler.start()
+            time.sleep(0.3)
         if dist is not None:
             dist.barrier()
-
-    # warm-up
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-
-    # timed region: exactly K replays of the step graph
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    total_ms = t0.elapsed_time(t1)
-    # keep the GPU busy while the sampler catches a few more readings
-    t_end = time.time() + 0.4
-    while time.time() < t_end:
-        graph.replay()
         torch.cuda.synchronize()
-    clocks = sampler.stop()
-    total_ms = max_over_ranks(total_ms, dist, dev)
-    step_ms = total_ms / args.steps
-
-    # per-stage breakdown (graph with captured timing events)
-    reps = max(3, min(args.steps, 10))
-    dec_us, sel_us, att_us, rect_us = [], [], [], []
-    for _ in range(reps):
-        graph_t.replay()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(steps):
+                graph.replay()
+            t1.record(stream)
         torch.cuda.synchronize()
-        for t in range(f):
+        if dist is not None:
+            dist.barrier()
+        total_ms = t0.elapsed_time(t1)
+        clocks = None
+        if sampler is not None:
+            # keep the GPU busy while the sampler catches a few more readings
+            t_end = time.time() + 0.4
+            while time.time() < t_end:
+                graph.replay()
+                torch.cuda.synchronize()
+            clocks = sampler.stop()
+        return total_ms, clocks
+    res["timed_region"] = timed_region
+
+    def breakdown():
+        reps = max(3, min(args.steps, 10))
+        dec_us, sel_us, att_us, rect_us = [], [], [], []
+        for _ in range(reps):
+            graph_t.replay()
+            torch.cuda.synchronize()
+            for t in range(f):
+                for li in range(L):
+                    e0, _, e2 = timing["dec"][t][li]
+                    dec_us.append(e0.elapsed_time(e2) * 1000.0)
             for li in range(L):
-                e0, _, e2 = timing["dec"][t][li]
-                dec_us.append(e0.elapsed_time(e2) * 1000.0)
-        for li in range(L):
-            a, b = timing["rect"][li]
-            rect_us.append(a.elapsed_time(b) * 1000.0)
-        graph_s.replay()
-        torch.cuda.synchronize()
-        for t in range(f):
-            for li in range(L):
-                e0, e1, e2 = timing_s["dec"][t][li]
-                sel_us.append(e0.elapsed_time(e1) * 1000.0)
-                att_us.append(e1.elapsed_time(e2) * 1000.0)
+                a, b = timing["rect"][li]
+                rect_us.append(a.elapsed_time(b) * 1000.0)
+            if graph_s is not None:
+                graph_s.replay()
+                torch.cuda.synchronize()
+                for t in range(f):
+                    for li in range(L):
+                        e0, e1, e2 = timing_s["dec"][t][li]
+                        sel_us.append(e0.elapsed_time(e1) * 1000.0)
+                        att_us.append(e1.elapsed_time(e2) * 1000.0)
+        return dec_us, sel_us, att_us, rect_us
 
     # the sparse decode calls alone and the dense (r = 1) arm, each as f * L
     # calls back to back in one CUDA graph: the method's gain over dense
@@ -345,62 +408,173 @@ def run_ours(args, rank, world, local_rank):
         q, kn, vn = dec_in[t]
         resa.decode_dense(q, kn, vn, ly["k"], ly["v"], ly["desc"], len_start + t + 1, 1.0,
                           outs[li], ws[li], lse=lses[li])
-    sparse_graph_us = graph_us(sparse_call)
-    dense_graph_us = graph_us(dense_call)
 
-    # the attention kernel on its own: f * L launches back to back (every
-    # layer's selected blocks, so consecutive launches read different caches)
-    graph_a = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_a, stream=stream):
-        for t in range(f):
-            q = dec_in[t][0]
-            for li, ly in enumerate(layers):
-                resa.attend_blocks(q, ly["k"], ly["v"], len_start + t + 1, sels[li][t], 1.0,
-                                   outs[li], ws[li], lse=lses[li])
-    graph_a.replay()
-    torch.cuda.synchronize()
-    ta0 = torch.cuda.Event(enable_timing=True)
-    ta1 = torch.cuda.Event(enable_timing=True)
-    reps_a = max(3, min(args.steps, 10))
-    with torch.cuda.stream(stream):
-        ta0.record(stream)
-        for _ in range(reps_a):
-            graph_a.replay()
-        ta1.record(stream)
-    torch.cuda.synchronize()
-    attend_launch_us = ta0.elapsed_time(ta1) * 1000.0 / (reps_a * f * L)
+    def attend_alone():
+        # f * L launches back to back (every layer's selected blocks, so
+        # consecutive launches read different caches)
+        ga = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ga, stream=stream):
+            for t in range(f):
+                q = dec_in[t][0]
+                for li, ly in enumerate(layers):
+                    resa.attend_blocks(q, ly["k"], ly["v"], len_start + t + 1, sels[li][t], 1.0,
+                                       outs[li], ws[li], lse=lses[li])
+        ga.replay()
+        torch.cuda.synchronize()
+        ta0 = torch.cuda.Event(enable_timing=True)
+        ta1 = torch.cuda.Event(enable_timing=True)
+        reps_a = max(3, min(args.steps, 10))
+        with torch.cuda.stream(stream):
+            ta0.record(stream)
+            for _ in range(reps_a):
+                ga.replay()
+            ta1.record(stream)
+        torch.cuda.synchronize()
+        del ga
+        return ta0.elapsed_time(ta1) * 1000.0 / (reps_a * f * L)
+
+    def summary():
+        """Per-call and back-to-back figures with their byte counts."""
+        hbm_peak, tf_peak, peak_kind = peaks()
+        dec_us, sel_us, att_us, rect_us = breakdown()
+        sparse_graph_us = graph_us(sparse_call)
+        dense_graph_us = graph_us(dense_call)
+        attend_launch_us = attend_alone()
+        for w in ws:
+            assert resa.workspace_status(w) == resa.RESA_OK
+        # bytes of the algorithm (descriptors + selected K/V + Q/O)
+        n_mid = n_at[f // 2]
+        len_mid = len_start + f // 2 + 1
+        M_mid = (len_mid + 15) // 16
+        qo = 2 * B * Hq * d * esize
+        desc_bytes = B * H * M_mid * 2 * d * esize
+        sel_kv = B * H * n_mid * 16 * 2 * d * esize
+        attend_bytes = sel_kv + qo + B * H * n_mid * 4
+        decode_bytes = desc_bytes + sel_kv + qo
+        rect_len = len_start + f
+        rect_bytes = (B * H * rect_len * 2 * d * esize + 2 * B * f * Hq * d * esize
+                      + 2 * B * f * H * d * esize)
+        rect_flops = 4.0 * B * Hq * d * (f * rect_len - f * (f - 1) / 2)
+        decode_med = statistics.median(dec_us)
+        rect_med = statistics.median(rect_us)
+        att_gbs = attend_bytes / (attend_launch_us * 1e-6) / 1e9
+        out = {
+            "decode_us": round(decode_med, 3),
+            "decode_us_p10_p90": [round(float(np.percentile(dec_us, 10)), 3),
+                                  round(float(np.percentile(dec_us, 90)), 3)],
+            "sparse_decode_graph_us": round(sparse_graph_us, 3),
+            "dense_decode_graph_us": round(dense_graph_us, 3),
+            "speedup_vs_dense": round(dense_graph_us / sparse_graph_us, 2),
+            "decode_bytes": decode_bytes,
+            "decode_hbm_gbs": round(decode_bytes / (decode_med * 1e-6) / 1e9, 1),
+            "decode_frac_of_measured_hbm": round(decode_bytes / (decode_med * 1e-6) / 1e9 / hbm_peak, 4),
+            "decode_graph_frac_of_measured_hbm": round(
+                decode_bytes / (sparse_graph_us * 1e-6) / 1e9 / hbm_peak, 4),
+            "attend_launch_us": round(attend_launch_us, 3),
+            "attend_hbm_gbs": round(att_gbs, 1),
+            "attend_frac_of_measured_hbm": round(att_gbs / hbm_peak, 4),
+            "attend_bytes": attend_bytes,
+            "rectify_us": round(rect_med, 3),
+            "rectify_amortised_us_per_token": round(rect_med / f, 3),
+            "rectify_hbm_gbs": round(rect_bytes / (rect_med * 1e-6) / 1e9, 1),
+            "rectify_frac_of_measured_hbm": round(rect_bytes / (rect_med * 1e-6) / 1e9 / hbm_peak, 4),
+            "rectify_tflops": round(rect_flops / (rect_med * 1e-6) / 1e12, 2),
+            "build_desc_us": round(build_desc_us, 2),
+        }
+        if sel_us:
+            out["staged_decode_us"] = round(statistics.median([a + b for a, b in zip(sel_us, att_us)]), 3)
+            out["staged_select_us"] = round(statistics.median(sel_us), 3)
+            out["staged_attend_us"] = round(statistics.median(att_us), 3)
+        return out
+    res["summary"] = summary
+
+    def e2e():
+        return run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt)
+    res["e2e"] = e2e
+    return res
+
+
+def extra_workloads(args, resa, dev, stream, L):
+    """The other benchmark workloads on the same GPU (amortised step, per-call
+    and back-to-back decode, attention alone, rectify, dense arm)."""
+    import torch
+    from workload import config
+    runs = [("resa_decode_256k_b1_r0.1", 3, {}), ("resa_decode_256k_b1_r0.05", 3, {"r": 0.05}),
+            ("resa_decode_32k_b4_needles", 1, {}), ("resa_decode_64k_b16_f32_r0.1", 4, {})]
+    out = {}
+    for name, idx, over in runs:
+        spec = config(idx, steps=64, **over)
+        m = measure_workload(args, resa, spec, L, dev, stream, host_cache=False, full=False)
+        total_ms, _ = m["timed_region"](max(3, args.steps // 4), args.warmup)
+        step_ms = total_ms / max(3, args.steps // 4)
+        s = m["summary"]()
+        s = {"value": round(step_ms * 1000.0 / (spec.f * L), 3), **s,
+             "amortised_speedup_vs_dense": round(s["dense_decode_graph_us"] /
+                                                 (step_ms * 1000.0 / (spec.f * L)), 2),
+             "context": spec.len0, "batch": spec.batch, "r": spec.r, "f": spec.f}
+        out[name] = s
+        del m
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import __graft_entry__
+    __graft_entry__.build()
+    import block_sparse_attention_quest_b200 as resa
+    from workload import config
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg_idx = WORKLOADS[args.workload]
+    over = {"steps": 64}
+    if args.r is not None:
+        over["r"] = args.r
+    if args.f is not None:
+        over["f"] = args.f
+    spec = config(cfg_idx, **over)
+    shard = args.shard == "heads" and world > 1
+    if shard:
+        # this rank's KV heads of every layer (no exchange inside the path)
+        import dataclasses
+        from block_sparse_attention_quest_b200.sharding import kv_head_range
+        h0, h1 = kv_head_range(spec.n_kv_heads, rank, world)
+        spec = dataclasses.replace(spec, n_kv_heads=h1 - h0, n_q_heads=(h1 - h0) * spec.group)
+    f, L = spec.f, args.layers
+    B, Hq, H = spec.batch, spec.n_q_heads, spec.n_kv_heads
+    stream = torch.cuda.Stream(device=dev)
+    m = measure_workload(args, resa, spec, L, dev, stream, host_cache=not shard, full=True)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    # timed region: exactly K replays of the step graph after W warm-up ones
+    total_ms, clocks = m["timed_region"](args.steps, args.warmup, dist, ClockSampler(local_rank))
+    total_ms = max_over_ranks(total_ms, dist, dev)
+    step_ms = total_ms / args.steps
+    summ = m["summary"]()
 
     # end-to-end through the public API with host buffers (eager calls)
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt)
+        e2e = m["e2e"]()
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
-
-    assert resa.workspace_status(ws[0]) == resa.RESA_OK
-    # bytes of the algorithm (descriptors + selected K/V + Q/O)
-    n_mid = n_at[f // 2]
-    len_mid = len_start + f // 2 + 1
-    M_mid = (len_mid + 15) // 16
-    qo = 2 * B * Hq * d * esize
-    desc_bytes = B * H * M_mid * 2 * d * esize
-    sel_kv = B * H * n_mid * 16 * 2 * d * esize
-    attend_bytes = sel_kv + qo + B * H * n_mid * 4
-    decode_bytes = desc_bytes + sel_kv + qo
-    rect_len = len_start + f
-    rect_bytes = B * H * rect_len * 2 * d * esize + 2 * B * f * Hq * d * esize + 2 * B * f * H * d * esize
-    rect_flops = 4.0 * B * Hq * d * (f * rect_len - f * (f - 1) / 2)
+        if world > 1:
+            e2e["h2d"] *= world
+            e2e["d2h"] *= world
 
     hbm_peak, tf_peak, peak_kind = peaks()
-    sel_med = statistics.median(sel_us)
-    att_med = statistics.median(att_us)
-    rect_med = statistics.median(rect_us)
-    decode_med = statistics.median(dec_us)
-    staged_med = statistics.median([a + b for a, b in zip(sel_us, att_us)])
-    dec_gbs = decode_bytes / (decode_med * 1e-6) / 1e9
-    att_gbs = attend_bytes / (attend_launch_us * 1e-6) / 1e9
-    us_per_decode = step_ms * 1000.0 / (f * L) / world
-    tokens_per_s = B * f * L * world / (step_ms * 1e-3) / L
+    # replicas: every rank decodes a whole layer; head shards: the ranks
+    # decode one layer together
+    units = 1 if shard else world
+    us_per_decode = step_ms * 1000.0 / (f * L) / units
+    tokens_per_s = B * f * L * units / (step_ms * 1e-3) / L
     launches_per_step = f * L * 3 + L * 3
+    wl = WORKLOAD_NAMES[cfg_idx]
+    custom = args.r is not None or args.f is not None
     res = {
         "metric": METRIC,
         "value": round(us_per_decode, 3),
@@ -410,51 +584,43 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup,
         "ms_per_step": round(step_ms, 4),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if shard else "weak",
         "vs_baseline": None,
         "dtype": spec.dtype,
         "data": "synthetic (seeded N(0,1) + block means; no dataset, no weights)",
         "config": {
-            "workload": WORKLOAD_NAMES[cfg_idx], "batch": B, "context": spec.len0,
-            "q_heads": Hq, "kv_heads": H, "head_dim": d, "block": 16, "r": spec.r,
+            "workload": wl, "batch": B, "context": spec.len0,
+            "q_heads": Hq, "kv_heads": H, "head_dim": spec.head_dim, "block": 16, "r": spec.r,
             "n_min": spec.n_min, "f": f, "layers": L,
             "step": f"{f} sparse decode steps x {L} layers + {L} rectifications",
             "l2": f"inputs larger than L2: {L} independent layer caches visited round-robin",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "parallelism": (f"KV-head shards x{world} (this rank's heads: {H})" if shard else
+                            f"replicas x{world}" if world > 1 else "single GPU"),
             "timing": "CUDA graph replay, CUDA events on the launching stream",
         },
-        "decode_us": round(decode_med, 3),
-        "decode_us_p10_p90": [round(float(np.percentile(dec_us, 10)), 3),
-                              round(float(np.percentile(dec_us, 90)), 3)],
-        "sparse_decode_graph_us": round(sparse_graph_us, 3),
-        "dense_decode_graph_us": round(dense_graph_us, 3),
-        "speedup_vs_dense": round(dense_graph_us / sparse_graph_us, 2),
-        "amortised_speedup_vs_dense": round(dense_graph_us / us_per_decode, 2),
+        **summ,
+        "amortised_speedup_vs_dense": round(summ["dense_decode_graph_us"] / us_per_decode, 2),
         "decode_kernels": "score_kernel -> select_reg_kernel -> attend_bf16_kernel (PDL chain)",
-        "staged_decode_us": round(staged_med, 3),
-        "staged_select_us": round(sel_med, 3),
-        "staged_attend_us": round(att_med, 3),
-        "attend_launch_us": round(attend_launch_us, 3),
-        "attend_hbm_gbs": round(att_gbs, 1),
-        "decode_hbm_gbs": round(decode_bytes / (decode_med * 1e-6) / 1e9, 1),
-        "decode_bytes": decode_bytes,
-        "decode_frac_of_measured_hbm": round(decode_bytes / (decode_med * 1e-6) / 1e9 / hbm_peak, 4),
-        "rectify_us": round(rect_med, 3),
-        "rectify_amortised_us_per_token": round(rect_med / f, 3),
-        "rectify_hbm_gbs": round(rect_bytes / (rect_med * 1e-6) / 1e9, 1),
-        "rectify_tflops": round(rect_flops / (rect_med * 1e-6) / 1e12, 2),
-        "build_desc_us": round(build_desc_us, 2),
         "tokens_per_s": round(tokens_per_s, 1),
         "roofline": {
             "kernel": "attend_bf16_kernel (split-KV attention, LSE merge in the last CTA)",
             "timing": "average over f * layers back-to-back launches in one CUDA graph",
-            "bound": "hbm", "achieved": round(att_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(att_gbs / hbm_peak, 4),
-            "traffic": (NCU_TRAFFIC.get(WORKLOAD_NAMES[cfg_idx])
-                        if args.r is None and args.f is None else None),
-            "peak_kind": f"{peak_kind} copy bandwidth",
-            "bytes_per_launch": attend_bytes,
+            "bound": "hbm", "achieved": summ["attend_hbm_gbs"], "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(summ["attend_hbm_gbs"] / hbm_peak, 4),
+            "traffic": None if custom else counter("attention", "traffic", wl),
+            "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+            "bytes_per_launch": summ["attend_bytes"],
             "bytes": "selected K/V + q + out + block ids",
+        },
+        "rectify": {
+            "kernel": "rectify_tc_kernel (tcgen05.mma, TMEM accumulators) + merge_rows_kernel",
+            "us": summ["rectify_us"], "hbm_gbs": summ["rectify_hbm_gbs"],
+            "frac_of_measured_hbm": summ["rectify_frac_of_measured_hbm"],
+            "tflops": summ["rectify_tflops"],
+            "tensor_pipe_active_pct": (None if custom or wl != "resa_decode_128k_b1"
+                                       else counter("rectify", "tensor_pipe_active_pct")),
+            "tensor_pipe_source": "ncu sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active, "
+                                  "one cold launch at 128K, f = 32 (null once the kernel changed)",
         },
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -462,9 +628,14 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_prefill:
         res["prefill"] = run_prefill(resa, stream, dev, tf_peak, peak_kind)
     if e2e is not None:
-        res["e2e"] = {"value": round(e2e["ms_per_step"] * 1000.0 / (f * L) / world, 3),
+        res["e2e"] = {"value": round(e2e["ms_per_step"] * 1000.0 / (f * L) / units, 3),
                       "unit": "us", "h2d_bytes_per_step": e2e["h2d"],
                       "d2h_bytes_per_step": e2e["d2h"]}
+    del m
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if not args.no_workloads and world == 1 and not custom and args.workload == "128k":
+        res["workloads"] = extra_workloads(args, resa, dev, stream, L)
     return res, spec
 
 
@@ -578,28 +749,49 @@ def run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, de
 
 
 # ----------------------------------------------------------------- CPU oracle
+def host_info() -> dict:
+    """Core count and CPU model of the host the oracle runs on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
 class OracleSample:
     """The CPU oracle on a bounded sample of the workload. One sample step is
     one decode step of the whole batch plus the rectification of one (batch,
-    KV head) group, the latter scaled by the number of groups; amortised over
-    f it gives microseconds per decode step in the benchmark's unit."""
+    KV head) group; the rectification time, scaled by the number of groups
+    and amortised over f, is added to the decode time to give microseconds
+    per amortised decode step (the benchmark's unit). The wall time of the
+    sample step itself is kept too."""
 
     def __init__(self, spec):
         import oracle as orc
         from workload import make_cache
         self.orc = orc
         self.spec = spec
-        try:
-            from threadpoolctl import threadpool_info
-            self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        except Exception:
-            self.threads = os.cpu_count() or 1
         K, V = make_cache(spec)
         self.st = orc.State(K, V, spec.len0, spec.group)
         self.groups = spec.batch * spec.n_kv_heads
         self.n = 0
 
+    @staticmethod
+    def threads() -> int:
+        """Threads the oracle's BLAS calls use under the current limits."""
+        try:
+            from threadpoolctl import threadpool_info
+            return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            return os.cpu_count() or 1
+
     def step(self):
+        """Returns (us per amortised decode step, wall seconds of the sample)."""
         from workload import decode_inputs, rectify_inputs
         spec, st, orc = self.spec, self.st, self.orc
         q, kn, vn = decode_inputs(spec, self.n % spec.steps)
@@ -614,14 +806,39 @@ class OracleSample:
         sub.length, sub.group = st.length, G
         t0 = time.perf_counter()
         sub.rectify(q_f[:1, :, :G], k_f[:1, :, :1], v_f[:1, :, :1], f, 1.0)
-        rect_s = (time.perf_counter() - t0) * self.groups
+        rect1_s = time.perf_counter() - t0
         self.n += 1
-        return (dec_s + rect_s / f) * 1e6
+        return (dec_s + rect1_s * self.groups / f) * 1e6, dec_s + rect1_s
 
     def describe(self, steps):
         return (f"{steps} sample steps, each = 1 oracle decode step (whole batch) + rectify of 1 "
-                f"of {self.groups} (batch, KV head) groups scaled x{self.groups}, amortised over "
-                f"f={self.spec.f}; context {self.spec.len0}")
+                f"of {self.groups} (batch, KV head) groups; value = decode + rectify x{self.groups} "
+                f"/ f={self.spec.f}; context {self.spec.len0}")
+
+    def timed(self, steps: int, single_thread: bool = False):
+        """Median us per amortised decode step and median sample wall ms over
+        `steps` sample steps (after one warm-up), on all cores or one."""
+        import contextlib
+        ctx = contextlib.nullcontext()
+        if single_thread:
+            from threadpoolctl import threadpool_limits
+            ctx = threadpool_limits(limits=1)
+        with ctx:
+            threads = self.threads()
+            self.step()
+            runs = [self.step() for _ in range(steps)]
+        return (statistics.median(r[0] for r in runs), statistics.median(r[1] for r in runs) * 1e3,
+                threads)
+
+
+def cpu_baseline(spec, steps: int = 3) -> dict:
+    """The oracle on this host, on all cores and on one thread."""
+    smp = OracleSample(spec)
+    us, _, threads = smp.timed(steps)
+    us1, _, _ = smp.timed(steps, single_thread=True)
+    return {"value": round(us, 1), "unit": "us", "cores": threads, "kind": "oracle",
+            "sample": smp.describe(steps), **host_info(),
+            "single_thread": {"value": round(us1, 1), "unit": "us", "cores": 1}}
 
 
 def run_reference(args, rank, world):
@@ -637,20 +854,25 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     smp = OracleSample(spec)
+    threads = smp.threads()
     for _ in range(args.warmup):
         smp.step()
-    per = [smp.step() for _ in range(args.steps)]
-    us = statistics.median(per)
+    runs = [smp.step() for _ in range(args.steps)]
+    us = statistics.median(r[0] for r in runs)
+    wall_ms = statistics.median(r[1] for r in runs) * 1e3
     return {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(us * spec.f * args.layers / 1000.0, 3),
+        "ms_per_step": round(wall_ms, 3),
+        "ms_per_step_is": "measured wall time of one sample step (1 decode + 1 group's rectify)",
+        "value_is": "us per amortised decode step computed from the sample "
+                    "(decode + rectify x groups / f)",
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) + block means; no dataset, no weights)",
         "config": {"workload": WORKLOAD_NAMES[cfg_idx], "batch": spec.batch,
                    "context": spec.len0, "r": spec.r, "f": spec.f, "layers": args.layers},
-        "cpu_baseline": {"value": round(us, 1), "unit": "us", "cores": smp.threads,
-                         "kind": "oracle", "sample": smp.describe(args.steps)},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us", "cores": threads,
+                         "kind": "oracle", "sample": smp.describe(args.steps), **host_info()},
         "e2e": {"value": round(us, 1), "unit": "us", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -675,12 +897,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res, spec = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = OracleSample(spec)
-        smp.step()                       # warm-up (page-in, BLAS threads)
-        per = [smp.step() for _ in range(3)]
-        res["cpu_baseline"] = {"value": round(statistics.median(per), 1), "unit": "us",
-                               "cores": smp.threads, "kind": "oracle",
-                               "sample": smp.describe(3)}
+        res["cpu_baseline"] = cpu_baseline(spec)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
