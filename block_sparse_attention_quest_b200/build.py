@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libresa.so")
-SOURCES = ["api.cu", "desc.cu", "select.cu", "attend.cu", "rectify_tc.cu", "noalloc.cu", "decode_fused.cu"]
+SOURCES = ["api.cu", "desc.cu", "select.cu", "attend.cu", "rectify_tc.cu", "noalloc.cu", "decode_coop.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

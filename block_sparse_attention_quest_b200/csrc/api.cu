@@ -72,6 +72,22 @@ bool make_cache_map(CUtensorMap* m, const void* base, const Shape& s, uint32_t b
   return r == CUDA_SUCCESS;
 }
 
+// 2-D view [B*H*Mmax*2 rows][D cols] of bf16 descriptors (min and max rows of
+// every block), 64 x 32 boxes without swizzle
+bool make_desc_map(CUtensorMap* m, const void* base, const Shape& s) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(s.D),
+                        static_cast<cuuint64_t>(s.B) * s.H * static_cast<cuuint64_t>(s.Mmax) * 2};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(s.D) * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 3-D view [B*f][Hq][D] of bf16 rectify queries; a (64 x G x 128/G) box is
 // one 128-row tile in the order row = query * G + head
 bool make_query_map(CUtensorMap* m, const void* base, const Shape& s, int f) {
@@ -124,13 +140,16 @@ int check_dims(const resa_dims* d, Shape* s) {
 
 int64_t blocks_of(int64_t len) { return (len + 15) / 16; }
 
-// The three-kernel decode step (score, select, attend, chained by
-// programmatic dependent launch) is the default. RESA_DECODE_FUSED=1 in the
-// environment selects the one-launch kernel for bf16 (decode_fused.cu); it
-// is exact as well, but its per-CTA redundant selection is slower today.
-bool fused_decode_enabled() {
+// Decode steps run as the three-kernel chain (score, select, attend, chained
+// by programmatic dependent launch). RESA_DECODE_ONE_LAUNCH=1 in the
+// environment runs bf16 steps at one length as one launch instead
+// (decode_coop.cu), where the shape allows it: the same step, measured slower
+// on B200 (its one CTA per SM streams the descriptors more slowly than the
+// score kernel, and its selection rounds through L2 cost more than the
+// chain's single-CTA selection).
+bool one_launch_enabled() {
   static const bool on = [] {
-    const char* e = std::getenv("RESA_DECODE_FUSED");
+    const char* e = std::getenv("RESA_DECODE_ONE_LAUNCH");
     return e != nullptr && e[0] == '1';
   }();
   return on;
@@ -153,8 +172,12 @@ int64_t split_bound(int64_t units) {
 }
 
 struct WsLayout {
-  size_t scores, sel, counters, part_ml, part_o, total;
+  size_t scores, sel, kept, counters, coop, part_ml, part_o, total;
 };
+
+bool coop_groups_fit(const Shape& s) {
+  return s.bf16 && static_cast<int64_t>(s.B) * s.H <= kCoopMaxGroups;
+}
 
 // Control block and arrival counters come first, at offsets that depend on
 // the dims only: they must stay put (and zero) from call to call. The scratch
@@ -165,10 +188,15 @@ WsLayout ws_layout(const Shape& s, int64_t len, int32_t f) {
   size_t off = kCtrlBytes;
   w.counters = off;
   off = align_up(off + static_cast<size_t>(s.B) * s.H * kMaxRectifyRows * sizeof(int));
+  // per-group state of the one-launch decode step (zero between calls)
+  w.coop = off;
+  if (coop_groups_fit(s)) off = align_up(off + static_cast<size_t>(s.B) * s.H * coop_group_bytes());
   w.scores = off;
   off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(float));
   w.sel = off;
   off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(int32_t));
+  w.kept = off;
+  if (coop_groups_fit(s)) off = align_up(off + static_cast<size_t>(s.B) * s.H * M * sizeof(int32_t));
   // decode rows: B*Hq with units B*H; rectify rows: B*f*Hq with units B*H*f
   const int64_t dec = static_cast<int64_t>(s.B) * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H);
   // a smaller window can take more splits, so size for the largest need of
@@ -362,30 +390,31 @@ static int decode_sparse_impl(const resa_dims* dims, const void* q, const void* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const WsLayout w = ws_layout(s, len, 0);
   int32_t* selp = sel ? sel : reinterpret_cast<int32_t*>(ws + w.sel);
-  if (s.bf16 && lens == nullptr && fused_decode_enabled()) {
-    // one launch: the CTAs of each KV group score, select and attend together
+  if (s.bf16 && lens == nullptr && one_launch_enabled() && coop_groups_fit(s)) {
+    // one launch: the CTAs of each KV group score their slices, agree on the
+    // exact top-n cut through the workspace and attend to equal shares
     const int num_sms = device_sms();
     if (num_sms <= 0) return RESA_ERR_CUDA;
-    const int groups = s.B * s.H;
-    int cpg = groups >= num_sms ? 1 : num_sms / groups;
-    if (cpg > kMaxSplits) cpg = kMaxSplits;
     const int M = static_cast<int>(blocks_of(len));
-    if (cpg > M) cpg = M;
-    while (cpg > 1 && (n + cpg - 1) / cpg > fused_max_share()) --cpg;
-    if (M - 1 <= fused_max_keys(s.D) && (n + cpg - 1) / cpg <= fused_max_share()) {
-      FusedLaunch f{};
-      f.s = s; f.q = q; f.k_new = k_new; f.v_new = v_new; f.k = k_cache; f.v = v_cache;
-      f.desc = desc; f.out = out; f.lse = lse; f.sel = sel;
-      f.scores = reinterpret_cast<float*>(ws + w.scores);
-      f.part_o = reinterpret_cast<float*>(ws + w.part_o);
-      f.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
-      f.sync = reinterpret_cast<int*>(ws + w.counters) + static_cast<int64_t>(groups);
-      f.ctrl = reinterpret_cast<Ctrl*>(ws);
-      f.len = len; f.M = M; f.n = n; f.cpg = cpg; f.scale = softmax_scale;
-      CUtensorMap tk, tv;
-      if (!make_cache_map(&tk, k_cache, s) || !make_cache_map(&tv, v_cache, s)) return RESA_ERR_CUDA;
-      f.tm_k = &tk; f.tm_v = &tv;
-      return cuda_status(launch_decode_fused(f, static_cast<cudaStream_t>(stream)));
+    const int S = splits_for(s.B * s.H, n, num_sms, s);
+    if (coop_supported(s, M, n, S)) {
+      CoopLaunch c{};
+      c.s = s; c.q = q; c.k_new = k_new; c.v_new = v_new; c.k = k_cache; c.v = v_cache;
+      c.desc = desc; c.out = out; c.lse = lse; c.sel = selp;
+      c.scores = reinterpret_cast<float*>(ws + w.scores);
+      c.kept = reinterpret_cast<int32_t*>(ws + w.kept);
+      c.groups = ws + w.coop;
+      c.part_o = reinterpret_cast<float*>(ws + w.part_o);
+      c.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+      c.counters = reinterpret_cast<int*>(ws + w.counters);
+      c.ctrl = reinterpret_cast<Ctrl*>(ws);
+      c.len = len; c.M = M; c.n = n; c.S = S; c.scale = softmax_scale;
+      CUtensorMap tk, tv, td;
+      if (!make_cache_map(&tk, k_cache, s) || !make_cache_map(&tv, v_cache, s) ||
+          !make_desc_map(&td, desc, s))
+        return RESA_ERR_CUDA;
+      c.tm_k = &tk; c.tm_v = &tv; c.tm_d = &td;
+      return cuda_status(launch_decode_coop(c, static_cast<cudaStream_t>(stream)));
     }
   }
   rc = select_impl(dims, q, k_new, v_new, k_cache, v_cache, desc, len, r, n_min, selp,

@@ -76,8 +76,9 @@ struct AttnArgs {
 };
 cudaError_t launch_attend(const Shape& s, const AttnArgs& a, cudaStream_t st);
 
-// one-launch decode step (bf16): score, select, attend, merge
-struct FusedLaunch {
+// one-launch decode step (bf16): append, score, cooperative exact top-n
+// selection, attention and merge (decode_coop.cu); S CTAs per KV group
+struct CoopLaunch {
   Shape s;
   const void* q;
   const void* k_new;
@@ -87,21 +88,27 @@ struct FusedLaunch {
   void* desc;
   void* out;
   float* lse;
-  int32_t* sel;
-  float* scores;
+  int32_t* sel;           // [B][H][n] list written by the step
+  float* scores;          // [B][H][M] workspace
+  int32_t* kept;          // [B][H][M] workspace
+  void* groups;           // [B*H] per-group state, zero between calls
   float* part_o;
   float* part_ml;
-  int* sync;              // [B*H][2], zero between calls
+  int* counters;          // [B*H] merge arrivals, zero between calls
   Ctrl* ctrl;
   int64_t len;
-  int M, n, cpg;
+  int M, n, S;
   float scale;
   const CUtensorMap* tm_k;
   const CUtensorMap* tm_v;
+  const CUtensorMap* tm_d;  // descriptors as [B*H*Mmax*2][D], 64 x 32 boxes
 };
-cudaError_t launch_decode_fused(const FusedLaunch& f, cudaStream_t st);
-int fused_max_keys(int D);
-int fused_max_share();
+cudaError_t launch_decode_coop(const CoopLaunch& c, cudaStream_t st);
+// whether the one-launch kernel takes M blocks, n selected, S CTAs per group
+bool coop_supported(const Shape& s, int M, int n, int S);
+// workspace bytes of one group's state (256-byte multiple)
+size_t coop_group_bytes();
+constexpr int kCoopMaxGroups = 64;   // groups (batch x KV heads) the one-launch path serves
 
 // rectification attention on tcgen05 (bf16, group size 1, 2, 4 or 8)
 struct RectArgs {

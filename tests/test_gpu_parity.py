@@ -340,16 +340,20 @@ def test_config_64k_batch16(r):
     _run_sampled(spec, steps=2, rect_f=(16, 32, 64) if r == 0.1 else (), rows=[0, 7, 15])
 
 
-def test_one_launch_decode_path():
-    """The one-launch decode kernel (selected by RESA_DECODE_FUSED=1), run in a
-    child process so that the choice does not leak into other tests."""
+@pytest.mark.parametrize("len0,batch", [(20000, 2), (131072, 1)])
+def test_one_launch_decode_path(len0, batch):
+    """The one-launch decode kernel (RESA_DECODE_ONE_LAUNCH=1: the CTAs of each
+    KV group score their slices, agree on the exact cut through the
+    workspace and attend to equal shares), run in a child process so that the
+    choice does not leak into other tests; also rows where every block is
+    kept and where only the newest one is."""
     import subprocess
     import sys
     code = (
         "import sys; sys.path.insert(0, '.');"
         "from tests.pair import Pair;"
         "from workload import Spec;"
-        "spec = Spec(batch=2, n_q_heads=32, n_kv_heads=8, head_dim=128, len0=20000, steps=6,"
+        f"spec = Spec(batch={batch}, n_q_heads=32, n_kv_heads=8, head_dim=128, len0={len0}, steps=4,"
         "            dtype='bf16', r=0.1, n_min=16);"
         "p = Pair(spec);"
         "[p.decode(s) for s in range(spec.steps)];"
@@ -357,13 +361,49 @@ def test_one_launch_decode_path():
         "spec2 = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=640, steps=2,"
         "             dtype='bf16', r=0.1, n_min=4);"
         "p2 = Pair(spec2); [p2.decode(s) for s in range(2)];"
+        "p3 = Pair(spec2, r=1.0); [p3.decode(s) for s in range(2)];"
+        "p4 = Pair(spec2, r=1e-4, n_min=1); [p4.decode(s) for s in range(2)];"
+        "spec5 = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, len0=16 * 3000, steps=2,"
+        "             dtype='bf16', r=0.1, n_min=4);"
+        "p5 = Pair(spec5); [p5.decode(s) for s in range(2)];"
         "print('one-launch ok')")
     import os
-    env = dict(os.environ, RESA_DECODE_FUSED="1")
+    env = dict(os.environ, RESA_DECODE_ONE_LAUNCH="1")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True,
-                       text=True, timeout=600)
-    assert r.returncode == 0 and "one-launch ok" in r.stdout, r.stdout + r.stderr
+                       text=True, timeout=900)
+    assert r.returncode == 0 and "one-launch ok" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+def test_one_launch_ties_and_crowded_bins():
+    """The one-launch kernel on rows whose threshold is an exact tie: every
+    block identical (one key), and three constant patterns (a crowded
+    threshold bin resolved by the radix passes)."""
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, '.');"
+        "import numpy as np;"
+        "from tests.pair import Pair;"
+        "from workload import Spec, make_cache, round_to;"
+        "spec = Spec(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, len0=16 * 3000, steps=2,"
+        "            dtype='bf16', r=0.1, n_min=4);"
+        "K, V = make_cache(spec); K[:] = round_to(np.full_like(K, 0.5), 'bf16');"
+        "p = Pair(spec, cache=(K, V)); res = [p.decode(s) for s in range(2)];"
+        "assert all(np.array_equal(r['gpu_sel'], r['sel']) for r in res);"
+        "K, V = make_cache(spec); rng = np.random.default_rng(99);"
+        "pats = round_to(rng.standard_normal((3, 128)).astype(np.float32), 'bf16');"
+        "which = rng.integers(0, 3, size=(1, 2, 3000));"
+        "K[:, :, :spec.len0] = np.repeat(pats[which], 16, axis=2);"
+        "p = Pair(spec, cache=(K, V)); res = [p.decode(s) for s in range(2)];"
+        "assert all(np.array_equal(r['gpu_sel'], r['sel']) for r in res);"
+        "print('ties ok')")
+    import os
+    env = dict(os.environ, RESA_DECODE_ONE_LAUNCH="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=900)
+    assert r.returncode == 0 and "ties ok" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 def test_back_to_back_calls_without_host_sync():
