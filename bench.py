@@ -49,10 +49,11 @@ METRIC = "ReSA decode-step us & achieved HBM GB/s vs roofline at 128K/256K; rect
 #   rectify: sm__pipe_tensor_cycles_active (% of peak, active cycles) of
 #     rectify_tc_kernel at 128K, f = 32 (--set full, one cold launch).
 NCU_COUNTERS = {
-    "attention": {"files": ["attend.cu", "common.cuh", "launch.h"], "source": None,
-                  "traffic": {"resa_decode_128k_b1": None}},
-    "rectify": {"files": ["rectify_tc.cu", "tc.cuh", "common.cuh", "launch.h"], "source": None,
-                "tensor_pipe_active_pct": None, "traffic": None},
+    "attention": {"files": ["attend.cu", "attend_core.cuh", "common.cuh", "launch.h"],
+                  "source": "1e1653cb0a1ec052",
+                  "traffic": {"resa_decode_128k_b1": 53972352}},
+    "rectify": {"files": ["rectify_tc.cu", "tc.cuh", "common.cuh", "launch.h"], "source": "47686c52fb77bf78",
+                "tensor_pipe_active_pct": 32.01, "traffic": 541409024},
 }
 
 
