@@ -200,14 +200,16 @@ WsLayout ws_layout(const Shape& s, int64_t len, int32_t f) {
   // decode rows: B*Hq with units B*H; rectify rows: B*f*Hq with units B*H*f
   const int64_t dec = static_cast<int64_t>(s.B) * s.Hq * split_bound(static_cast<int64_t>(s.B) * s.H);
   // a smaller window can take more splits, so size for the largest need of
-  // every window up to f
+  // every window up to f (none for a decode-only workspace, f = 0)
   int64_t rec = 0;
-  for (int64_t fr = 1; fr <= (f > 0 ? f : 1); ++fr) {
-    int64_t sb = split_bound(static_cast<int64_t>(s.B) * s.H * fr);
-    const int64_t sb_tc = split_bound(static_cast<int64_t>(s.B) * s.H * rect_mtiles(s, static_cast<int>(fr)));
-    if (sb_tc > sb) sb = sb_tc;
+  for (int64_t fr = 1; fr <= f; ++fr) {
+    const int64_t sb = split_bound(static_cast<int64_t>(s.B) * s.H * fr);
     const int64_t need = static_cast<int64_t>(s.B) * fr * s.Hq * sb;
     if (need > rec) rec = need;
+    // tensor-core path: 128 rows per (batch row, KV head, m-tile) and split
+    const int64_t tc_units = static_cast<int64_t>(s.B) * s.H * rect_mtiles(s, static_cast<int>(fr));
+    const int64_t need_tc = tc_units * 128 * split_bound(tc_units);
+    if (need_tc > rec) rec = need_tc;
   }
   const int64_t rows = dec > rec ? dec : rec;
   w.part_ml = off;
@@ -530,6 +532,7 @@ static int rectify_impl(const resa_dims* dims, const void* q_f, const void* k_f,
         !make_cache_map(&tv, v_cache, s, 128))
       return RESA_ERR_CUDA;
     r.tm_q = &tq; r.tm_k = &tk; r.tm_v = &tv;
+    r.pdl = true;
     return cuda_status(launch_rectify_tc(r, st));
   }
   return run_attention(s, q_f, f, len - f + 1, nullptr, 0, softmax_scale, k_cache, v_cache, out_f,

@@ -226,6 +226,20 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 }
 // Bring a contiguous global range into L2 (16-byte aligned start, size a
 // multiple of 16); returns no data, so it may precede a dependency wait.
+// Bulk copy shared -> global (both 16-byte aligned, bytes a multiple of 16)
+// in this thread's bulk group; bulk_commit closes the group and
+// bulk_wait_read blocks until every committed group has read its source.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(dst), "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }

@@ -8,6 +8,8 @@
 //
 // All three kernels are bound by HBM traffic of the keys they read; the
 // min/max of bf16 values is exact in float and converts back exactly.
+#include <atomic>
+
 #include "launch.h"
 
 namespace resa {
@@ -103,6 +105,9 @@ __global__ void rectify_write_kernel(const T* __restrict__ k_f, const T* __restr
                                      T* __restrict__ k, T* __restrict__ v, T* __restrict__ desc,
                                      int H, int D, int64_t L_max, int Mmax, int64_t len, int f,
                                      const int32_t* lens, const int32_t* windows, Ctrl* ctrl) {
+  // the attention over the rectified rows may launch now: its CTAs wait for
+  // this grid before reading any row written here
+  grid_launch_dependents();
   const int c = threadIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * H + h;
@@ -117,19 +122,30 @@ __global__ void rectify_write_kernel(const T* __restrict__ k_f, const T* __restr
   if (j * kBlock >= len) return;           // this row touches fewer blocks
   const int64_t t0 = j * kBlock;
   const int64_t t1 = t0 + kBlock < len ? t0 + kBlock : len;
-  float mn = INFINITY, mx = -INFINITY;
-  for (int64_t t = t0; t < t1; ++t) {
-    T kv;
+  // every load of the block is issued before the first store
+  T kv[kBlock], vv[kBlock];
+#pragma unroll
+  for (int i = 0; i < kBlock; ++i) {
+    const int64_t t = t0 + i;
+    if (t >= t1) continue;
     if (t >= t_first) {
-      const int64_t i = t - t_first;
-      const int64_t src = ((static_cast<int64_t>(b) * f + i) * H + h) * D + c;
-      kv = k_f[src];
-      k[(bh * L_max + t) * D + c] = kv;
-      v[(bh * L_max + t) * D + c] = v_f[src];
+      const int64_t src = ((static_cast<int64_t>(b) * f + (t - t_first)) * H + h) * D + c;
+      kv[i] = k_f[src];
+      vv[i] = v_f[src];
     } else {
-      kv = k[(bh * L_max + t) * D + c];
+      kv[i] = k[(bh * L_max + t) * D + c];
     }
-    const float x = Dt<T>::to_f(kv);
+  }
+  float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kBlock; ++i) {
+    const int64_t t = t0 + i;
+    if (t >= t1) continue;
+    if (t >= t_first) {
+      k[(bh * L_max + t) * D + c] = kv[i];
+      v[(bh * L_max + t) * D + c] = vv[i];
+    }
+    const float x = Dt<T>::to_f(kv[i]);
     mn = fminf(mn, x);
     mx = fmaxf(mx, x);
   }
@@ -186,6 +202,24 @@ cudaError_t launch_rectify_write(const Shape& s, const void* k_f, const void* v_
   const int64_t M = (len + kBlock - 1) / kBlock;
   const int64_t touched = (lens || windows) ? f / kBlock + 2 : M - j0;
   dim3 grid(static_cast<unsigned>(touched), s.H, s.B);
+  // The attention over the rectified rows, launched next, takes nearly all
+  // of an SM's shared memory and may start while this grid runs: with the
+  // same (maximal) shared-memory carveout its CTAs can start on the SMs this
+  // grid occupies instead of waiting for them to drain.
+  static std::atomic<bool> carveout_set[64][2];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!carveout_set[dev][s.bf16]) {
+    cudaError_t e = s.bf16 ? cudaFuncSetAttribute(rectify_write_kernel<__nv_bfloat16>,
+                                                  cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                  cudaSharedmemCarveoutMaxShared)
+                           : cudaFuncSetAttribute(rectify_write_kernel<float>,
+                                                  cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                  cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    carveout_set[dev][s.bf16] = true;
+  }
   if (s.bf16) {
     using T = __nv_bfloat16;
     rectify_write_kernel<T><<<grid, s.D, 0, st>>>(

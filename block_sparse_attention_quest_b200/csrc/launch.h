@@ -120,12 +120,14 @@ struct RectArgs {
   void* desc;             // prefill (f = len, S = 1): descriptors written from the K tiles
   float scale;
   void* out;              // [B][f][Hq][D] bf16
-  float* part_o;          // [B*f*Hq][S][D]
-  float* part_ml;         // [B*f*Hq][S][2]
+  float* part_o;          // [S][B*H*mtiles][128][D] (S > 1), float4 units swizzled per row
+  float* part_ml;         // [S][B*H*mtiles][128][2]
   Ctrl* ctrl;
   const CUtensorMap* tm_q;  // q_f as [B*f][Hq][D], 64 x G x (128/G) boxes
   const CUtensorMap* tm_k;  // cache as [B*H*L_max][D], 64 x 128 boxes
   const CUtensorMap* tm_v;
+  bool pdl;               // launched right after the rectify write kernel: CTAs that
+                          // do not read the rewritten rows start before it ends
 };
 cudaError_t launch_rectify_tc(const RectArgs& r, cudaStream_t st);
 int attend_ctas_per_sm(const Shape& s);

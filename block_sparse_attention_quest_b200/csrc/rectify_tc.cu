@@ -29,6 +29,14 @@
 // Keys past the end of the cache (the padded tail of the last tile) are
 // masked in S and their V rows are zeroed in shared memory before the PV
 // product, so stale cache contents never reach an output.
+//
+// In a rectification the kernel is launched as a programmatic dependent of
+// the kernel that writes the f new rows into the cache: only the CTAs whose
+// key range reaches those rows wait for it before their first copy, the rest
+// start streaming at once. The split merge is launched the same way and
+// waits for this grid before reading the partials.
+#include <type_traits>
+
 #include "launch.h"
 #include "tc.cuh"
 
@@ -36,8 +44,8 @@ namespace resa {
 
 struct RectK {
   void* out;             // [B][f][Hq][D] bf16 (used when S == 1)
-  float* part_o;         // [B*f*Hq][S][D]
-  float* part_ml;        // [B*f*Hq][S][2]
+  float* part_o;         // [S][units][128][D], each row's float4 units swizzled
+  float* part_ml;        // [S][units][128][2]
   Ctrl* ctrl;
   int64_t len;
   int64_t L_max;
@@ -45,7 +53,7 @@ struct RectK {
   const int32_t* windows;  // optional per-row windows [B] in [0, f]
   __nv_bfloat16* desc;   // prefill: descriptors of the queries' own tokens, or nullptr
   int64_t Mmax;
-  int B, H, Hq, G, f, S, mtiles;
+  int B, H, Hq, G, f, S, mtiles;   // units = B * H * mtiles: (b, g, m-tile) = unit
   float scale_log2;
 };
 
@@ -80,7 +88,6 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   __shared__ __align__(8) uint64_t bar_vfull[C::kStages], bar_vempty[C::kStages];
   __shared__ __align__(8) uint64_t bar_s[2], bar_p[2], bar_pv[2];
   __shared__ uint32_t tmem_base_sh;
-  __shared__ float s_m1[128], s_l1[128];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = base;
@@ -95,8 +102,14 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t len = row_len(a.lens, a.len, b);
   const int win = row_window(a.windows, a.f, b);   // query rows in use: 0 .. win-1
-  if (win == 0 || len < win) return;       // not rectified: skipped
-  if (mt * 128 >= win * a.G) return;       // this m-tile holds no row in use
+  // Launched after the kernel that writes the rectified rows into the cache
+  // (programmatic dependent launch): a CTA waits for it before reading any
+  // of those rows, and before it exits in any case (no-op otherwise).
+  if (win == 0 || len < win || mt * 128 >= win * a.G) {   // not rectified, or no row in use
+    grid_dependency_wait();
+    return;
+  }
+  grid_launch_dependents();
   // positions of this m-tile's first and last query rows; keys past the last
   // are masked for every row, so their tiles are not visited
   const int64_t qpos_lo = len - win + (mt * 128) / a.G;
@@ -145,7 +158,14 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
         tma_load_3d(sQ + hf * C::kHalfBytes, &tmQ, hf * 64, g * a.G, b * a.f + mt * rows_per_q,
                     &bar_q);
       const int64_t row0 = (static_cast<int64_t>(b) * a.H + g) * a.L_max;
+      // rows from len - win on are rewritten by the kernel this one may
+      // overlap: the first copy of a tile that reaches them waits for it
+      bool waited = false;
       auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int t) {
+        if (!waited && static_cast<int64_t>(t0 + t + 1) * 128 > len - win) {
+          grid_dependency_wait();
+          waited = true;
+        }
         const int y = static_cast<int>(row0 + static_cast<int64_t>(t0 + t) * 128);
         mbar_arrive_expect_tx(bar, C::kKBytes);
 #pragma unroll
@@ -220,7 +240,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
     const int w = warp >> 2;                               // warpgroup: tiles t = w (mod 2)
     const int row = threadIdx.x & 127;                     // TMEM lane / tile row
     const int rg = mt * 128 + row;
-    const int qi = rg / a.G, hh = rg % a.G;
+    const int qi = rg / a.G;
     const int64_t qpos = len - win + qi;                   // causal limit of this row
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
@@ -236,18 +256,33 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       // the cache) exist only in the last tiles
       const bool masked = key0 + 127 > qpos_lo;
       const int lim = masked ? static_cast<int>(qpos - key0 < 127 ? qpos - key0 : 127) : 127;
-      // pass 1: row maximum of the raw scores
-      float mx = -INFINITY;
+      // masked keys become -inf, which the exponential below turns into 0
+      auto mask = [&](float (&x)[32], int c4) {
+        if (masked) {
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tc::ld32(tS(w) + lane_off + c4 * 32, v);
+          for (int i = 0; i < 32; ++i)
+            if (c4 * 32 + i > lim) x[i] = -INFINITY;
+        }
+      };
+      // pass 1: row maximum as eight independent chains (a single chain of
+      // 128 dependent maxima is latency-bound)
+      float va[2][32];
+      float mp[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mp[j] = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tc::ld32(tS(w) + lane_off + 64 * h, va[0]);
+        tc::ld32(tS(w) + lane_off + 64 * h + 32, va[1]);
         tc::wait_ld();
+        mask(va[0], 2 * h);
+        mask(va[1], 2 * h + 1);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (!masked || c4 * 32 + i <= lim) mx = fmaxf(mx, v[i]);
+        for (int i = 0; i < 32; ++i) mp[i & 7] = fmaxf(mp[i & 7], fmaxf(va[0][i], va[1][i]));
       }
-      mx *= sl2;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) mp[j] = fmaxf(mp[j], mp[j + 4]);
+      float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * sl2;
       if (u > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_pv[w], (u - 1) & 1, a.ctrl));
         if (!ok) break;
@@ -277,22 +312,19 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       // 16 c4 .. 16 c4 + 15 of S (keys 32 c4 .. 32 c4 + 31): below the columns
       // still to be read, above none the A operand needs later
       const bool live = m_ref != -INFINITY;
+      const float nm = live ? -m_ref : 0.f;
       float sum = 0.f;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tc::ld32(tS(w) + lane_off + c4 * 32, v);
+        float x[32];
+        tc::ld32(tS(w) + lane_off + c4 * 32, x);
         tc::wait_ld();
+        mask(x, c4);
         uint32_t wd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c = c4 * 32 + 2 * e;
-          float p0 = ex2(fmaf(v[2 * e], sl2, -m_ref));
-          float p1 = ex2(fmaf(v[2 * e + 1], sl2, -m_ref));
-          if (masked) {
-            if (c > lim) p0 = 0.f;
-            if (c + 1 > lim) p1 = 0.f;
-          }
+          float p0 = ex2(fmaf(x[2 * e], sl2, nm));
+          float p1 = ex2(fmaf(x[2 * e + 1], sl2, nm));
           if (!live) { p0 = 0.f; p1 = 0.f; }
           sum += p0 + p1;
           wd[e] = pack_bf16x2(p0, p1);
@@ -304,12 +336,12 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       // V rows past the end of the cache are zeroed (0 * stale data must not
       // reach an output)
       if (key0 + row >= len) {
-        uint8_t* v = sV(t % C::kStages);
+        uint8_t* vt = sV(t % C::kStages);
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf)
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(v + hf * C::kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vt + hf * C::kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
@@ -352,16 +384,21 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       // the group has read it first
       if (w == 1) asm volatile("bar.sync 2, 128;" ::: "memory");
     }
-    // combine the two warpgroups: group 1 hands (m, l, O) over through the
-    // K/V stage of its last tile, idle once that tile's PV product has
+    // combine the two warpgroups: group 1 hands O over through the K/V
+    // stage of its last tile, idle once that tile's PV product has
     // completed (no copy targets it afterwards, and group 0's remaining tile
     // uses another stage); with no tile of its own, through stage 1, which
-    // is never loaded then
+    // is never loaded then. A row's D values sit in its own D * 4 bytes of
+    // the stage as float4 units, unit j at j ^ (row mod D/4): conflict-free
+    // both for one thread per row and for one warp per row.
+    constexpr int NJ = D / 4;                                // float4 units per row
     const int t_last1 = (nt & 1) ? nt - 2 : nt - 1;          // last odd tile
-    float* sO1 = reinterpret_cast<float*>(sK(nt >= 2 ? t_last1 % C::kStages : 1));
+    float4* sO1 = reinterpret_cast<float4*>(sK(nt >= 2 ? t_last1 % C::kStages : 1));
+    auto slot = [&](int r, int j) { return r * NJ + (j ^ (r & (NJ - 1))); };
     if (w == 1) {
-      s_m1[row] = has ? m_ref : -INFINITY;
-      s_l1[row] = has ? l : 0.f;
+      // (m, l) of the row go to the first two columns of the group's S block,
+      // unused once its last PV product has completed
+      tc::st2(tS(1) + lane_off, has ? m_ref : -INFINITY, has ? l : 0.f);
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         float o[32];
@@ -373,19 +410,27 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sO1[row * D + ((c4 * 32 + i + row) % D)] = o[i];
+        for (int k = 0; k < 8; ++k)
+          sO1[slot(row, c4 * 8 + k)] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
       }
     }
+    if (w == 1) tc::wait_st();
+    tc::fence_before_sync();
     asm volatile("bar.sync 1, 256;" ::: "memory");
+    tc::fence_after_sync();
     if (w == 0 && ok) {
-      const float m1 = s_m1[row], l1 = s_l1[row];
+      float m1, l1;
+      tc::ld2(tS(1) + lane_off, m1, l1);
+      tc::wait_ld();
       const float m0 = has ? m_ref : -INFINITY, l0 = has ? l : 0.f;
       const float m = fmaxf(m0, m1);
       const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
       const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
       const float lt = a0 * l0 + a1 * l1;
-      const bool valid = qi < win;
-      const int64_t orow = (static_cast<int64_t>(b) * a.f + qi) * a.Hq + g * a.G + hh;
+      // the combined row replaces group 1's in the stage (normalised when it
+      // is the final output) ...
+      const float sc = a.S == 1 ? 1.f / lt : 1.f;
+      const float b0 = a0 * sc, b1 = a1 * sc;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         float o[32];
@@ -396,26 +441,52 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
+        // all eight units are read before any is written back (the
+        // compiler cannot tell the slots apart, so interleaved they would
+        // serialise on shared-memory latency)
+        float4 y[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = a0 * o[i] + a1 * sO1[row * D + ((c4 * 32 + i + row) % D)];
-        if (valid) {
-          if (a.S == 1) {
-            const float inv = 1.f / lt;
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + orow * D + c4 * 32;
+        for (int k = 0; k < 8; ++k) y[k] = sO1[slot(row, c4 * 8 + k)];
 #pragma unroll
-            for (int i = 0; i < 32; i += 2)
-              *reinterpret_cast<uint32_t*>(dst + i) = pack_bf16x2(o[i] * inv, o[i + 1] * inv);
-          } else {
-            float* dst = a.part_o + (orow * a.S + s_idx) * D + c4 * 32;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-          }
-        }
+        for (int k = 0; k < 8; ++k)
+          sO1[slot(row, c4 * 8 + k)] =
+              make_float4(b0 * o[4 * k] + b1 * y[k].x, b0 * o[4 * k + 1] + b1 * y[k].y,
+                          b0 * o[4 * k + 2] + b1 * y[k].z, b0 * o[4 * k + 3] + b1 * y[k].w);
       }
-      if (valid && a.S > 1) {
-        a.part_ml[(orow * a.S + s_idx) * 2] = m;
-        a.part_ml[(orow * a.S + s_idx) * 2 + 1] = lt;
+      // (each warp's lanes wrote exactly the 32 rows the warp stores below)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (a.S > 1) {
+        // ... and a split's partial rows of this unit form one contiguous
+        // block of the workspace, copied as the stage holds it (rows past
+        // the window included; the merge never reads them): one bulk copy
+        // of 32 rows per warp
+        const int64_t unit = (static_cast<int64_t>(b) * a.H + g) * a.mtiles + mt;
+        const int64_t prow = (s_idx * static_cast<int64_t>(a.B) * a.H * a.mtiles + unit) * 128;
+        reinterpret_cast<float2*>(a.part_ml)[prow + row] = make_float2(m, lt);
+        if (lane == 0) {
+          const int r0 = (warp & 3) * 32;
+          bulk_store(a.part_o + (prow + r0) * D, sO1 + r0 * NJ, 32 * D * 4);
+          bulk_commit();
+          bulk_wait_read();
+        }
+        __syncwarp();
+      } else {
+        // ... and each warp writes its 32 rows out whole (32 / NJ rows per
+        // store instruction, each a contiguous run of global memory)
+        constexpr int RPI = 32 / NJ;
+        const int j = lane % NJ;
+#pragma unroll 4
+        for (int it = 0; it < 32 / RPI; ++it) {
+          const int r = (warp & 3) * 32 + it * RPI + lane / NJ;
+          const int rgr = mt * 128 + r;
+          const int qr = rgr / a.G;
+          if (qr >= win) continue;
+          const int64_t orow = (static_cast<int64_t>(b) * a.f + qr) * a.Hq + g * a.G + rgr % a.G;
+          const float4 x = sO1[slot(r, j)];
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + orow * D + 4 * j) =
+              make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+        }
       }
     }
   }
@@ -425,64 +496,84 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
     tc::fence_after_sync();
     tc::dealloc(tmem, C::kTmemCols);
   }
+  grid_dependency_wait();
 }
 
-// Merge of split partials for independent rows: one warp per row.
+// Merge of split partials for independent rows: one warp per output row,
+// each lane owning D/32 of its columns. Split s of the unit (b, g, m-tile)
+// holding tile row r left (m, l) at part_ml[(s * units + unit) * 128 + r] and
+// its D values at the same row of part_o, float4 unit j at position
+// j ^ (r mod D/4). The merge runs online over groups of up to 32 splits
+// (running maximum, rescaled sum), so every load of a group is issued before
+// any is used and no separate pass over the maxima comes first.
 template <int D>
 __global__ void __launch_bounds__(128) merge_rows_kernel(const float* __restrict__ part_o,
                                                          const float* __restrict__ part_ml,
                                                          __nv_bfloat16* __restrict__ out,
-                                                         int64_t rows, int S,
+                                                         int64_t rows, int S, int64_t units,
                                                          const int32_t* lens, int64_t len,
-                                                         const int32_t* windows,
-                                                         int64_t rows_per_b, int f, int Hq) {
+                                                         const int32_t* windows, int f, int H,
+                                                         int Hq, int G, int mtiles) {
   constexpr int CPL = D / 32;
+  constexpr int NJ = D / 4;
+  using Vec = typename std::conditional<CPL == 4, float4, float2>::type;
+  // the partials come from the previous kernel (programmatic dependent launch)
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
+  const int64_t rows_per_b = static_cast<int64_t>(f) * Hq;
+  const int b = static_cast<int>(row / rows_per_b);
+  const int qi = static_cast<int>((row % rows_per_b) / Hq);
+  const int h = static_cast<int>(row % Hq);
   if (lens != nullptr || windows != nullptr) {
-    const int b = static_cast<int>(row / rows_per_b);
     const int w = row_window(windows, f, b);
-    const int qi = static_cast<int>((row % rows_per_b) / Hq);
     if (qi >= w || row_len(lens, len, b) < w) return;   // row not rectified
   }
-  const float* ml = part_ml + row * S * 2;
-  float mstar = -INFINITY;
-  for (int s = lane; s < S; s += 32) mstar = fmaxf(mstar, ml[2 * s]);
-  mstar = warp_max_xor(mstar, 16, 1);
-  float lsum = 0.f;
-  for (int s = lane; s < S; s += 32) {
-    const float m = ml[2 * s];
-    lsum += m == -INFINITY ? 0.f : exp2f(m - mstar) * ml[2 * s + 1];
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  const int rg = qi * G + h % G;                         // row within the unit's tiles
+  const int r = rg & 127;
+  const int64_t unit = (static_cast<int64_t>(b) * H + h / G) * mtiles + (rg >> 7);
+  // this lane's columns: float4 unit j (whole for D = 128, half for D = 64)
+  const int j = lane * CPL / 4;
+  const int col = ((j ^ (r & (NJ - 1))) * 4) + (lane * CPL) % 4;
+  const float2* ml = reinterpret_cast<const float2*>(part_ml) + unit * 128 + r;
+  const float* po = part_o + (unit * 128 + r) * D + col;
+  const int64_t split_rows = units * 128;                 // rows between splits
+  float m_run = -INFINITY, l_run = 0.f;
   float acc[CPL];
 #pragma unroll
   for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
-  const float* po = part_o + row * S * D + lane * CPL;
-  int s = 0;
-  for (; s + 4 <= S; s += 4) {
-    float w[4], x[4][CPL];
+  for (int s0 = 0; s0 < S; s0 += 32) {
+    const int ns = S - s0 < 32 ? S - s0 : 32;
+    // lane u holds (m, l) of split s0 + u; every lane loads its columns of
+    // all the group's splits before any is used
+    const float2 p = lane < ns ? ml[(s0 + lane) * split_rows] : make_float2(-INFINITY, 0.f);
+    Vec x[32];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float m = ml[2 * (s + u)];
-      w[u] = m == -INFINITY ? 0.f : exp2f(m - mstar);
+    for (int u = 0; u < 32; ++u)
+      if (u < ns) x[u] = *reinterpret_cast<const Vec*>(po + (s0 + u) * split_rows * D);
+    const float m_new = fmaxf(m_run, warp_max_xor(p.x, 16, 1));
+    if (m_new == -INFINITY) continue;                    // no live split yet
+    const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+    const float w = p.x == -INFINITY ? 0.f : exp2f(p.x - m_new);
+    float wl = w * p.y;
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) x[u][i] = po[static_cast<int64_t>(s + u) * D + i];
+    for (int o = 16; o >= 1; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
+    l_run = fmaf(l_run, alpha, wl);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) acc[i] *= alpha;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const float wu = __shfl_sync(0xffffffffu, w, u);
+      if (u < ns) {
+        const float* xv = reinterpret_cast<const float*>(&x[u]);
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) acc[i] = fmaf(wu, xv[i], acc[i]);
+      }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w[u], x[u][i], acc[i]);
+    m_run = m_new;
   }
-  for (; s < S; ++s) {
-    const float m = ml[2 * s];
-    const float w = m == -INFINITY ? 0.f : exp2f(m - mstar);
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w, po[static_cast<int64_t>(s) * D + i], acc[i]);
-  }
-  const float inv = 1.f / lsum;
+  const float inv = 1.f / l_run;
   __nv_bfloat16* orow = out + row * D + lane * CPL;
 #pragma unroll
   for (int i = 0; i < CPL; ++i) orow[i] = __float2bfloat16_rn(acc[i] * inv);
@@ -499,6 +590,11 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(rectify_tc_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
+    // the merge is launched while this kernel runs: with the same carveout
+    // its CTAs can wait on SMs that still hold a CTA of this kernel
+    e = cudaFuncSetAttribute(merge_rows_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   RectK k{};
@@ -507,15 +603,31 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   k.lens = r.lens; k.windows = r.windows;
   k.desc = static_cast<__nv_bfloat16*>(r.desc); k.Mmax = r.L_max / 16; k.B = r.B;
   k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
-  dim3 grid(r.S, r.H, r.B * r.mtiles);
-  rectify_tc_kernel<D><<<grid, 288, C::kSmem, st>>>(*r.tm_q, *r.tm_k, *r.tm_v, k);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(r.S, r.H, r.B * r.mtiles);
+  cfg.blockDim = dim3(288);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = r.pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D>, *r.tm_q, *r.tm_k, *r.tm_v, k);
   if (e != cudaSuccess || r.S == 1) return e;
+  // the merge overlaps its launch with the rectify kernel's tail
   const int64_t rows = static_cast<int64_t>(r.B) * r.f * r.Hq;
-  merge_rows_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(
-      r.part_o, r.part_ml, static_cast<__nv_bfloat16*>(r.out), rows, r.S, r.lens, r.len,
-      r.windows, static_cast<int64_t>(r.f) * r.Hq, r.f, r.Hq);
-  return cudaGetLastError();
+  cudaLaunchConfig_t mcfg = {};
+  mcfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  mcfg.blockDim = dim3(128);
+  mcfg.stream = st;
+  mcfg.attrs = attr;
+  mcfg.numAttrs = 1;
+  const int64_t units = static_cast<int64_t>(r.B) * r.H * r.mtiles;
+  return cudaLaunchKernelEx(&mcfg, merge_rows_kernel<D>, static_cast<const float*>(r.part_o),
+                            static_cast<const float*>(r.part_ml),
+                            static_cast<__nv_bfloat16*>(r.out), rows, r.S, units, r.lens, r.len,
+                            r.windows, r.f, r.H, r.Hq, r.G, r.mtiles);
 }
 
 cudaError_t launch_rectify_tc(const RectArgs& r, cudaStream_t st) {

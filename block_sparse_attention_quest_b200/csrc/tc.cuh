@@ -131,6 +131,20 @@ __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t (&v)[16]) {
         "r"(v[14]), "r"(v[15])
       : "memory");
 }
+// two consecutive 32-bit columns of this thread's TMEM lane
+__device__ __forceinline__ void st2(uint32_t taddr, float a, float b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};"
+               ::"r"(taddr), "r"(__float_as_uint(a)), "r"(__float_as_uint(b))
+               : "memory");
+}
+__device__ __forceinline__ void ld2(uint32_t taddr, float& a, float& b) {
+  uint32_t r0, r1;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(taddr));
+  a = __uint_as_float(r0);
+  b = __uint_as_float(r1);
+}
 __device__ __forceinline__ void wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
