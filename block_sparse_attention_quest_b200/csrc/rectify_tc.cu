@@ -95,10 +95,15 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
   auto sK = [&](int st) { return sStage + st * C::kStageBytes; };
   auto sV = [&](int st) { return sStage + st * C::kStageBytes + C::kKBytes; };
 
-  // grid z runs over (m-tile, batch row) with the m-tiles that see the most
-  // keys first
-  const int s_idx = blockIdx.x, g = blockIdx.y;
-  const int b = blockIdx.z % a.B, mt = a.mtiles - 1 - static_cast<int>(blockIdx.z / a.B);
+  // Prefill: grid z runs over (m-tile, batch row) with the m-tiles that see
+  // the most keys first. Rectification: grid x runs over (m-tile, split)
+  // with the m-tile fastest, so the m-tiles of one split, which stream the
+  // same key tiles, run side by side and the second read of a tile hits L2.
+  const bool prefill = a.desc != nullptr;
+  const int s_idx = prefill ? blockIdx.x : blockIdx.x / a.mtiles, g = blockIdx.y;
+  const int b = prefill ? blockIdx.z % a.B : blockIdx.z;
+  const int mt = prefill ? a.mtiles - 1 - static_cast<int>(blockIdx.z / a.B)
+                         : static_cast<int>(blockIdx.x % a.mtiles);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t len = row_len(a.lens, a.len, b);
   const int win = row_window(a.windows, a.f, b);   // query rows in use: 0 .. win-1
@@ -607,7 +612,8 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(r.S, r.H, r.B * r.mtiles);
+  cfg.gridDim = r.desc != nullptr ? dim3(r.S, r.H, r.B * r.mtiles)
+                                   : dim3(r.S * r.mtiles, r.H, r.B);
   cfg.blockDim = dim3(288);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
