@@ -129,6 +129,7 @@ struct RectArgs {
   bool pdl;               // launched right after the rectify write kernel: CTAs that
                           // do not read the rewritten rows start before it ends
 };
+// dense rectification / prefill, then the split merge
 cudaError_t launch_rectify_tc(const RectArgs& r, cudaStream_t st);
 int attend_ctas_per_sm(const Shape& s);
 

@@ -57,6 +57,30 @@ struct RectK {
   float scale_log2;
 };
 
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// A staged output row of D fp32 values occupies its own D * 4 bytes as D/4
+// float4 units, unit j of row r at j ^ (r mod D/4): conflict-free both when
+// one thread writes its own row and when one warp reads a whole row. The
+// split partials keep this order in global memory (the merge undoes it).
+template <int D>
+__device__ __forceinline__ int stage_slot(int r, int j) {
+  constexpr int NJ = D / 4;
+  return r * NJ + (j ^ (r & (NJ - 1)));
+}
+
+// First row of the partials of split s for unit (b, g, m-tile).
+__device__ __forceinline__ int64_t partial_row(const RectK& a, int s, int b, int g, int mt) {
+  const int64_t units = static_cast<int64_t>(a.B) * a.H * a.mtiles;
+  const int64_t unit = (static_cast<int64_t>(b) * a.H + g) * a.mtiles + mt;
+  return (s * units + unit) * 128;
+}
+
+
 template <int D>
 struct RectCfg {
   static constexpr int kHalves = D / 64;
@@ -66,15 +90,13 @@ struct RectCfg {
   // K/V ring: tile t uses stage t % kStages (P lives in tensor memory)
   static constexpr int kStages = 3;
   static constexpr int kStageBytes = 2 * kKBytes;
-  static constexpr int kSmem = kQBytes + kStages * kStageBytes + 1024;
+  // at least 116 KB, so that one CTA fits an SM: a second would wait in
+  // its tensor-memory allocation for the first one's 512 columns
+  static constexpr int kSmem = kQBytes + kStages * kStageBytes + 1024 > 116 * 1024
+                                   ? kQBytes + kStages * kStageBytes + 1024
+                                   : 116 * 1024;
   static constexpr uint32_t kTmemCols = 512;              // S0 S1 O0 O1, 128 columns each
 };
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 template <int D>
 __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -339,14 +361,21 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
       tc::wait_st();
       l += sum;
       // V rows past the end of the cache are zeroed (0 * stale data must not
-      // reach an output)
-      if (key0 + row >= len) {
-        uint8_t* vt = sV(t % C::kStages);
+      // reach an output), once the tile's V copy, which may still be in
+      // flight when its S is ready, has landed
+      if (key0 + 127 >= len) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bar_vfull[t % C::kStages],
+                                                       (t / C::kStages) & 1, a.ctrl));
+        if (!ok) break;
+        if (key0 + row >= len) {
+          uint8_t* vt = sV(t % C::kStages);
 #pragma unroll
-        for (int hf = 0; hf < C::kHalves; ++hf)
+          for (int hf = 0; hf < C::kHalves; ++hf)
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(vt + hf * C::kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(vt + hf * C::kHalfBytes + row * 128 + c * 16) =
+                  make_uint4(0, 0, 0, 0);
+        }
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
@@ -399,7 +428,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
     constexpr int NJ = D / 4;                                // float4 units per row
     const int t_last1 = (nt & 1) ? nt - 2 : nt - 1;          // last odd tile
     float4* sO1 = reinterpret_cast<float4*>(sK(nt >= 2 ? t_last1 % C::kStages : 1));
-    auto slot = [&](int r, int j) { return r * NJ + (j ^ (r & (NJ - 1))); };
+    auto slot = [](int r, int j) { return stage_slot<D>(r, j); };
     if (w == 1) {
       // (m, l) of the row go to the first two columns of the group's S block,
       // unused once its last PV product has completed
@@ -466,8 +495,7 @@ __global__ void __launch_bounds__(288, 1) rectify_tc_kernel(const __grid_constan
         // block of the workspace, copied as the stage holds it (rows past
         // the window included; the merge never reads them): one bulk copy
         // of 32 rows per warp
-        const int64_t unit = (static_cast<int64_t>(b) * a.H + g) * a.mtiles + mt;
-        const int64_t prow = (s_idx * static_cast<int64_t>(a.B) * a.H * a.mtiles + unit) * 128;
+        const int64_t prow = partial_row(a, s_idx, b, g, mt);
         reinterpret_cast<float2*>(a.part_ml)[prow + row] = make_float2(m, lt);
         if (lane == 0) {
           const int r0 = (warp & 3) * 32;
@@ -570,7 +598,7 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const float* __restrict
 #pragma unroll
     for (int u = 0; u < 32; ++u) {
       const float wu = __shfl_sync(0xffffffffu, w, u);
-      if (u < ns) {
+      if (u < ns && wu != 0.f) {                        // (a split without keys adds nothing)
         const float* xv = reinterpret_cast<const float*>(&x[u]);
 #pragma unroll
         for (int i = 0; i < CPL; ++i) acc[i] = fmaf(wu, xv[i], acc[i]);
@@ -584,6 +612,50 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const float* __restrict
   for (int i = 0; i < CPL; ++i) orow[i] = __float2bfloat16_rn(acc[i] * inv);
 }
 
+// The merge is launched as a programmatic dependent of the rectification
+// kernel (it waits for that grid before reading the partials), so its launch
+// overlaps the kernel's tail; with the same shared-memory carveout its CTAs
+// can wait on SMs that still hold a rectification CTA.
+template <int D>
+static cudaError_t merge_rows_t(const RectArgs& r, cudaStream_t st) {
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(merge_rows_kernel<D>,
+                                         cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int64_t rows = static_cast<int64_t>(r.B) * r.f * r.Hq;
+  cudaLaunchConfig_t mcfg = {};
+  mcfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  mcfg.blockDim = dim3(128);
+  mcfg.stream = st;
+  mcfg.attrs = attr;
+  mcfg.numAttrs = 1;
+  const int64_t units = static_cast<int64_t>(r.B) * r.H * r.mtiles;
+  return cudaLaunchKernelEx(&mcfg, merge_rows_kernel<D>, static_cast<const float*>(r.part_o),
+                            static_cast<const float*>(r.part_ml),
+                            static_cast<__nv_bfloat16*>(r.out), rows, r.S, units, r.lens, r.len,
+                            r.windows, r.f, r.H, r.Hq, r.G, r.mtiles);
+}
+
+static RectK rect_kernel_args(const RectArgs& r) {
+  RectK k{};
+  k.out = r.out; k.part_o = r.part_o; k.part_ml = r.part_ml; k.ctrl = r.ctrl;
+  k.len = r.len; k.L_max = r.L_max; k.H = r.H; k.Hq = r.Hq; k.G = r.G; k.f = r.f; k.S = r.S;
+  k.lens = r.lens; k.windows = r.windows;
+  k.desc = static_cast<__nv_bfloat16*>(r.desc); k.Mmax = r.L_max / 16; k.B = r.B;
+  k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
+  return k;
+}
+
 template <int D>
 static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   using C = RectCfg<D>;
@@ -595,19 +667,9 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(rectify_tc_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    // the merge is launched while this kernel runs: with the same carveout
-    // its CTAs can wait on SMs that still hold a CTA of this kernel
-    e = cudaFuncSetAttribute(merge_rows_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  RectK k{};
-  k.out = r.out; k.part_o = r.part_o; k.part_ml = r.part_ml; k.ctrl = r.ctrl;
-  k.len = r.len; k.L_max = r.L_max; k.H = r.H; k.Hq = r.Hq; k.G = r.G; k.f = r.f; k.S = r.S;
-  k.lens = r.lens; k.windows = r.windows;
-  k.desc = static_cast<__nv_bfloat16*>(r.desc); k.Mmax = r.L_max / 16; k.B = r.B;
-  k.mtiles = r.mtiles; k.scale_log2 = r.scale * 1.4426950408889634f;
+  const RectK k = rect_kernel_args(r);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -621,19 +683,7 @@ static cudaError_t rectify_tc_t(const RectArgs& r, cudaStream_t st) {
   cfg.numAttrs = r.pdl ? 1 : 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, rectify_tc_kernel<D>, *r.tm_q, *r.tm_k, *r.tm_v, k);
   if (e != cudaSuccess || r.S == 1) return e;
-  // the merge overlaps its launch with the rectify kernel's tail
-  const int64_t rows = static_cast<int64_t>(r.B) * r.f * r.Hq;
-  cudaLaunchConfig_t mcfg = {};
-  mcfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
-  mcfg.blockDim = dim3(128);
-  mcfg.stream = st;
-  mcfg.attrs = attr;
-  mcfg.numAttrs = 1;
-  const int64_t units = static_cast<int64_t>(r.B) * r.H * r.mtiles;
-  return cudaLaunchKernelEx(&mcfg, merge_rows_kernel<D>, static_cast<const float*>(r.part_o),
-                            static_cast<const float*>(r.part_ml),
-                            static_cast<__nv_bfloat16*>(r.out), rows, r.S, units, r.lens, r.len,
-                            r.windows, r.f, r.H, r.Hq, r.G, r.mtiles);
+  return merge_rows_t<D>(r, st);
 }
 
 cudaError_t launch_rectify_tc(const RectArgs& r, cudaStream_t st) {

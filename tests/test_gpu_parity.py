@@ -326,7 +326,8 @@ def test_config_32k_batch4_needles():
 
 
 def test_config_128k():
-    _run_sampled(config(2), steps=3, rect_f=(32,))
+    # f = 64: 256 query rows per KV head, two m-tiles
+    _run_sampled(config(2), steps=3, rect_f=(32, 64))
 
 
 @pytest.mark.parametrize("r", [0.1, 0.05])
