@@ -50,10 +50,10 @@ METRIC = "ReSA decode-step us & achieved HBM GB/s vs roofline at 128K/256K; rect
 #     rectify_tc_kernel at 128K, f = 32 (--set full, one cold launch).
 NCU_COUNTERS = {
     "attention": {"files": ["attend.cu", "attend_core.cuh", "common.cuh", "launch.h"],
-                  "source": "1e1653cb0a1ec052",
-                  "traffic": {"resa_decode_128k_b1": 53972352}},
-    "rectify": {"files": ["rectify_tc.cu", "tc.cuh", "common.cuh", "launch.h"], "source": "47686c52fb77bf78",
-                "tensor_pipe_active_pct": 32.01, "traffic": 541409024},
+                  "source": "21102da51ec3d8a4",
+                  "traffic": {"resa_decode_128k_b1": 53964672}},
+    "rectify": {"files": ["rectify_tc.cu", "tc.cuh", "common.cuh", "launch.h"], "source": "32e588cf2e8f88a6",
+                "tensor_pipe_active_pct": 36.22, "traffic": 544848384},
 }
 
 
