@@ -97,9 +97,11 @@ typedef struct {
 RESA_API int32_t resa_num_selected(int64_t len, int32_t block_size, double r, int32_t n_min);
 
 /* Workspace bytes that suffice for resa_decode_sparse, resa_decode_dense and
- * resa_rectify (with any window f' <= f) at any length up to `len`, and for
- * the *_varlen calls with len_bound <= len. Returns 0 for invalid dims, len < 1
- * or f outside [0, 256]. */
+ * resa_rectify (with any window 1 <= f' <= f) at any length up to `len`, and
+ * for the *_varlen calls with len_bound <= len. f = 0 sizes a workspace for
+ * the decode and prefill calls only (a rectification given one returns
+ * RESA_ERR_WORKSPACE). Returns 0 for invalid dims, len < 1 or f outside
+ * [0, 256]. */
 RESA_API size_t resa_workspace_bytes(const resa_dims* dims, int64_t len, int32_t f);
 
 /* Quest block descriptors of the first `len` tokens (per-block, per-channel

@@ -187,6 +187,21 @@ def test_workspace_covers_every_smaller_window(resa):
             assert resa.workspace_bytes(d, 4000, f) <= big, (kw, f)
 
 
+def test_decode_only_workspace_does_not_serve_a_rectification(resa):
+    """A workspace sized for decoding only (f = 0) holds no room for the
+    rectification's split partials: it is smaller than one sized for f = 1,
+    and a rectification given one is rejected before anything is launched."""
+    d = _dims(resa)
+    dec = resa.workspace_bytes(d, 4000, 0)
+    assert 0 < dec < resa.workspace_bytes(d, 4000, 1) <= resa.workspace_bytes(d, 4000, 32)
+    rc = resa._lib.resa_rectify(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4000, 32, 1.0,
+                                FAKE, FAKE, dec, None)
+    assert rc == resa.RESA_ERR_WORKSPACE
+    # two 128-row tiles per KV head (f = 64, 4 query heads per KV head) need
+    # room for the partials of both
+    assert resa.workspace_bytes(d, 4000, 64) >= resa.workspace_bytes(d, 4000, 32)
+
+
 def test_prefill_rejects_invalid_arguments(resa):
     E = resa
     lib = resa._lib
