@@ -637,6 +637,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.empty_cache()
     if not args.no_workloads and world == 1 and not custom and args.workload == "128k":
         res["workloads"] = extra_workloads(args, resa, dev, stream, L)
+        res["workloads"]["resa_decode_ragged_b4"] = run_varlen(resa, stream, dev, hbm_peak)
     return res, spec
 
 
@@ -675,6 +676,76 @@ def run_prefill(resa, stream, dev, tf_peak, peak_kind, length=16384):
             "peak": tf_peak, "peak_kind": f"{peak_kind} cuBLAS bf16 (burst)",
             "flops": flops, "bound": "tensor",
             "note": "descriptors of the prompt written by the same pass"}
+
+
+def run_varlen(resa, stream, dev, hbm_peak, lens=(131072, 98304, 65536, 32768), r=0.1,
+               n_min=16, f=32, windows=(32, 0, 17, 32)):
+    """A ragged batch (continuous batching): one cache length per row, each
+    row's descriptors, selection and attention bounded by its own length, and
+    a rectification with a window per row (0 = the row is not rectified).
+    CUDA events around back-to-back calls of the per-row-length entry points;
+    bytes = each row's descriptors + selected K/V + q/out (decode) and each
+    rectified row's whole cache (rectify)."""
+    import torch
+    B, Hq, H, d = len(lens), 32, 8, 128
+    max_len = ((max(lens) + 15) // 16) * 16 + 64
+    g = torch.Generator(device=dev).manual_seed(20240610)
+    k = torch.randn(B, H, max_len, d, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, max_len, d, device=dev, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, Hq, d, device=dev, generator=g).to(torch.bfloat16)
+    q_f = torch.randn(B, f, Hq, d, device=dev, generator=g).to(torch.bfloat16)
+    k_f = torch.randn(B, f, H, d, device=dev, generator=g).to(torch.bfloat16)
+    v_f = torch.randn(B, f, H, d, device=dev, generator=g).to(torch.bfloat16)
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=dev)
+    win_t = torch.tensor(windows, dtype=torch.int32, device=dev)
+    bound = max(lens)
+    desc = torch.zeros(B, H, max_len // 16, 2, d, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
+    out_f = torch.empty(B, f, Hq, d, dtype=torch.bfloat16, device=dev)
+    dims = resa.dims_for(k, Hq)
+    ws = resa.alloc_workspace(dims, max_len, f, device=dev)
+
+    def timed(call, reps):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                call()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                call()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1000.0 / reps
+
+    with torch.cuda.stream(stream):
+        resa.build_desc_varlen(k, lens_t, bound, desc, Hq, stream=stream)
+    dec_us = timed(lambda: resa.decode_sparse_varlen(q, None, None, k, v, desc, lens_t, bound, r,
+                                                     n_min, 1.0, out, ws, stream=stream), 64)
+    rect_us = timed(lambda: resa.rectify_varlen(q_f, k_f, v_f, k, v, desc, lens_t, bound, f, 1.0,
+                                                out_f, ws, windows=win_t, stream=stream), 8)
+    assert resa.workspace_status(ws) == resa.RESA_OK
+    esize = 2
+    dec_bytes = 2 * B * Hq * d * esize
+    rect_bytes = 0
+    for L_b, w_b in zip(lens, windows):
+        M = (L_b + 15) // 16
+        n = resa.num_selected(L_b, r, n_min)
+        dec_bytes += H * ((M - 1) * 2 * d * esize + n * 16 * 2 * d * esize)
+        if w_b > 0:
+            rect_bytes += H * L_b * 2 * d * esize + 2 * w_b * (Hq + H) * d * esize
+    del k, v, desc, ws
+    torch.cuda.empty_cache()
+    dec_gbs = dec_bytes / (dec_us * 1e-6) / 1e9
+    rect_gbs = rect_bytes / (rect_us * 1e-6) / 1e9
+    return {"lens": list(lens), "r": r, "n_min": n_min, "f": f, "windows": list(windows),
+            "decode_us": round(dec_us, 3), "decode_bytes": dec_bytes,
+            "decode_hbm_gbs": round(dec_gbs, 1), "decode_frac_of_measured_hbm": round(dec_gbs / hbm_peak, 4),
+            "rectify_us": round(rect_us, 3), "rectify_bytes": rect_bytes,
+            "rectify_hbm_gbs": round(rect_gbs, 1),
+            "rectify_frac_of_measured_hbm": round(rect_gbs / hbm_peak, 4),
+            "timing": "CUDA events around back-to-back calls of resa_decode_sparse_varlen and "
+                      "resa_rectify_varlen (no append, fixed lengths)"}
 
 
 def run_e2e(args, resa, spec, layers, ws, dec_in, rect_in, len_start, stream, dev, tdt):
